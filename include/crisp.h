@@ -1,0 +1,156 @@
+/*
+ * crisp.h -- C ABI of the CRISP sparse-prefill attention library (B200, sm_100a).
+ *
+ * CRISP ("Cliff-awaRe Input-adaptive Sparse Prefilling with
+ * Structural-Mass-Motivated Routing") prefills one attention layer in three
+ * stages per query head (CRISP paper summary page, Methodology and
+ * "Algorithm Overview", Algorithms 1-4):
+ *
+ *   1. proxy map A-hat: the last |Q-hat| = 64 queries scored against every
+ *      key, causal softmax taken after the scores (Algorithm 2);
+ *   2. route: C_struct = mean post-softmax mass on S_anchor (first w_sink
+ *      keys plus the w_local-key recency window), Eq. (2); the head goes to
+ *      Vertical-Slash (VS) if C_struct >= tau_proxy, else to pooled
+ *      estimation (PE);
+ *   3. selection: VS keeps column blocks and diagonal (offset) blocks whose
+ *      mass p_j exceeds alpha * mu, the sink-aware noise floor of Eq. (3)-(4),
+ *      always keeping the first and last block (Algorithm 3); PE pools Q and
+ *      K per block, scores the block map by softmax and keeps the smallest
+ *      gamma-cumulative set of blocks (Algorithm 4). Then exact causal
+ *      attention over exactly the selected keys (Algorithm 1).
+ *
+ * Tensors (all device memory, batch 1, head-major, contiguous, row-major):
+ *   q, out : [h_q ][n][d]      k, v : [h_kv][n][d]
+ * element type bf16 or fp32 (cfg.dtype); out has the same type as q.
+ * Query head h reads KV head h / (h_q / h_kv) (grouped-query attention).
+ * Blocks: B = cfg.block = 128 keys; N_b = n / B; W = ceil(N_b / 32).
+ *
+ * Conventions
+ * - Every entry point validates its arguments before it launches anything;
+ *   a failed validation returns an error and leaves memory untouched.
+ * - No entry point synchronises with the host, allocates memory or keeps
+ *   global mutable state. All scratch lives in the caller's workspace
+ *   (cfg.workspace, >= crisp_workspace_size bytes of device memory, 256-byte
+ *   aligned). Calls that share a workspace must be ordered (same stream).
+ * - `stream` is a cudaStream_t passed as a plain pointer (NULL = legacy
+ *   default stream). All work is enqueued on it.
+ * - Conditions found on the device (a bounded wait that ran out, a
+ *   non-finite proxy statistic) never trap: they set the workspace status
+ *   word, which crisp_device_status reads. Each entry point clears the
+ *   status word when it starts, so it reports on the most recent call.
+ * - Host-side launch failures return CRISP_ERR_CUDA.
+ */
+#ifndef CRISP_H
+#define CRISP_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  CRISP_OK = 0,
+  CRISP_ERR_INVALID_ARG = 1,   /* null pointer, non-finite or out-of-range knob */
+  CRISP_ERR_SHAPE = 2,         /* n, h_q, h_kv, d outside what this build supports */
+  CRISP_ERR_DTYPE = 3,         /* unknown element type */
+  CRISP_ERR_ALIGN = 4,         /* a tensor or workspace pointer not 16/256-byte aligned */
+  CRISP_ERR_WORKSPACE = 5,     /* workspace missing or smaller than crisp_workspace_size */
+  CRISP_ERR_UNSUPPORTED = 6,   /* a knob value the kernels do not implement */
+  CRISP_ERR_CUDA = 7,          /* a CUDA runtime call or launch failed */
+  CRISP_ERR_CAPACITY = 8,      /* device-side: an internal buffer would overflow */
+  CRISP_ERR_TIMEOUT = 9,       /* device-side: a bounded wait ran out */
+  CRISP_ERR_NONFINITE = 10     /* device-side: a proxy statistic was NaN or infinite */
+} crisp_status;
+
+typedef enum { CRISP_BF16 = 0, CRISP_FP32 = 1 } crisp_dtype;
+
+typedef enum { CRISP_ROUTE_AUTO = -1, CRISP_ROUTE_VS = 0, CRISP_ROUTE_PE = 1 } crisp_route_t;
+
+/* Layer shape and the method's knobs. Defaults are set by crisp_cfg_init. */
+typedef struct {
+  int32_t n;            /* sequence length; this build: multiple of 128, 512 <= n <= 1048576 */
+  int32_t h_q;          /* query heads */
+  int32_t h_kv;         /* key/value heads; h_q % h_kv == 0, h_q / h_kv <= 16 */
+  int32_t d;            /* head dimension; this build: 128 */
+  int32_t dtype;        /* crisp_dtype */
+  int32_t block;        /* B, block size of the partition (summary page, Eq. (3) text): 128 */
+  int32_t last_q;       /* |Q-hat|, proxy query rows (Algorithm 2): 64 */
+  int32_t w_sink;       /* sink window of S_anchor (Eq. (2) text): 128 */
+  int32_t w_local;      /* recency window of S_anchor (Eq. (2) text): 128 */
+  float tau_proxy;      /* route threshold of C_struct; the pages give no value: default 0.10 */
+  float alpha;          /* Eq. (4) multiplier on the noise floor; default 1.0; >= 0 */
+  float gamma;          /* PE cumulative coverage (Algorithm 4); default 0.95; in (0, 1] */
+  float sm_scale;       /* softmax scale; <= 0 means 1/sqrt(d) */
+  int32_t force_route;  /* crisp_route_t: -1 route by C_struct, 0 force VS, 1 force PE */
+  int32_t reserved;     /* must be 0 */
+  void* workspace;      /* device scratch owned by the caller */
+  size_t workspace_bytes;
+} crisp_cfg;
+
+/* Selection outputs; every pointer is a caller-owned device buffer.
+ * Bit b of a mask lives in word b / 32, bit position b % 32. */
+typedef struct {
+  int32_t* route;       /* [h_q]           0 = VS, 1 = PE */
+  float* c_struct;      /* [h_q]           Eq. (2) */
+  float* p_v;           /* [h_q][N_b]      column-block masses (sum over each block of the column means) */
+  float* p_s;           /* [h_q][N_b]      offset-block masses (diagonal i - j in [bB, bB+B)) */
+  float* mu;            /* [h_q][2]        noise floors (mu_v, mu_s), Eq. (3) */
+  uint32_t* vs_mask;    /* [h_q][2][W]     selected column blocks, then selected offset blocks */
+  int32_t* v_idx;       /* [h_q][N_b]      selected column blocks, ascending, first nv[h] valid */
+  int32_t* s_idx;       /* [h_q][N_b]      selected offset blocks, ascending, first ns[h] valid */
+  int32_t* nv;          /* [h_q] */
+  int32_t* ns;          /* [h_q] */
+  uint32_t* pe_mask;    /* [h_q][N_b][W]   PE block mask, row = query block; valid where route == PE */
+  int64_t* pe_count;    /* [h_q]           selected causal blocks of the PE mask (0 for VS heads) */
+  float* pe_cut;        /* [h_q]           normalised value of the last block kept by the gamma cut
+                                           (0 when every block is kept or the head is VS) */
+} crisp_index;
+
+/* Fill *cfg with the defaults above for the given shape (workspace NULL). */
+crisp_status crisp_cfg_init(crisp_cfg* cfg, int32_t n, int32_t h_q, int32_t h_kv, int32_t d, int32_t dtype);
+
+/* Bytes of workspace the calls below need for cfg's shape. */
+crisp_status crisp_workspace_size(const crisp_cfg* cfg, size_t* bytes);
+
+/* Number of 32-bit words W per mask row, and N_b, for cfg's shape. */
+crisp_status crisp_index_dims(const crisp_cfg* cfg, int32_t* n_blocks, int32_t* words);
+
+/* Algorithm 2 (PatSearch): proxy map, C_struct (Eq. (2)) and the route of
+ * every query head. Writes route[h_q] and c_struct[h_q] (device). */
+crisp_status crisp_route(const void* q, const void* k, const crisp_cfg* cfg,
+                         int32_t* route, float* c_struct, void* stream);
+
+/* Algorithms 2-4: route and the selected index sets of every head. */
+crisp_status crisp_select(const void* q, const void* k, const crisp_cfg* cfg,
+                          const crisp_index* index, void* stream);
+
+/* Algorithm 1's last step: causal attention over the keys the given index
+ * selects (index->route, vs_mask and pe_mask are read, nothing else). */
+crisp_status crisp_attend(const void* q, const void* k, const void* v, void* out,
+                          const crisp_cfg* cfg, const crisp_index* index, void* stream);
+
+/* Algorithm 1: route, select and sparse attention for the whole layer. */
+crisp_status crisp_prefill(const void* q, const void* k, const void* v, void* out,
+                           const crisp_cfg* cfg, void* stream);
+
+/* Exact dense causal attention with the same kernels (the speed reference). */
+crisp_status crisp_dense_attention(const void* q, const void* k, const void* v, void* out,
+                                   const crisp_cfg* cfg, void* stream);
+
+/* Synchronise `stream`, then read (and clear) the workspace status word.
+ * *device_status receives a crisp_status code (CRISP_OK if none). */
+crisp_status crisp_device_status(const crisp_cfg* cfg, void* stream, int32_t* device_status);
+
+/* Short English description of a status code (static storage). */
+const char* crisp_status_string(crisp_status status);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int32_t crisp_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CRISP_H */

@@ -1,0 +1,362 @@
+// C ABI of the CRISP sparse-prefill library: argument validation, workspace
+// layout and the order of kernel launches. Nothing here synchronises with the
+// device except crisp_device_status.
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <algorithm>
+
+#include "crisp.h"
+#include "internal.h"
+
+namespace crisp {
+
+static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+WsLayout ws_layout(const Shape& s) {
+  WsLayout L;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align256(off + bytes);
+    return o;
+  };
+  const size_t hq = s.h_q, hkv = s.h_kv, nb = s.nb, rows = (size_t)s.h_q * s.last_q;
+  L.status = take(256);
+  L.part_lo = take(rows * nb * 4);
+  L.part_hi = take(rows * nb * 4);
+  L.chunk_ml = take(rows * s.n_chunks * 8);
+  L.chunk_w = take(rows * s.n_chunks * 4);
+  L.tile_a = take(hq * nb * 4);
+  L.tile_b = take(hq * nb * 4);
+  L.qbar = take(hq * nb * kHeadDim * 4);
+  L.kbar = take(hkv * nb * kHeadDim * 4);
+  L.tri = take(hq * (size_t)s.tri * 4);
+  L.hist = take(hq * sizeof(PeHist));
+  L.pe_state = take(hq * sizeof(PeState));
+  L.tie_rows = take(hq * nb * 4);
+  L.kv_pe = take(hkv * 4);
+  L.route = take(hq * 4);
+  L.c_struct = take(hq * 4);
+  L.p_v = take(hq * nb * 4);
+  L.p_s = take(hq * nb * 4);
+  L.mu = take(hq * 2 * 4);
+  L.vs_mask = take(hq * 2 * (size_t)s.words * 4);
+  L.v_idx = take(hq * nb * 4);
+  L.s_idx = take(hq * nb * 4);
+  L.nv = take(hq * 4);
+  L.ns = take(hq * 4);
+  L.pe_mask = take(hq * nb * (size_t)s.words * 4);
+  L.pe_count = take(hq * 8);
+  L.pe_cut = take(hq * 4);
+  L.total = off;
+  return L;
+}
+
+bool use_tensor_cores() {
+  const char* e = getenv("CRISP_FORCE_SIMT");
+  return !(e && e[0] == '1');
+}
+
+static IndexPtrs internal_index(char* ws, const WsLayout& L) {
+  IndexPtrs p;
+  p.route = reinterpret_cast<int32_t*>(ws + L.route);
+  p.c_struct = reinterpret_cast<float*>(ws + L.c_struct);
+  p.p_v = reinterpret_cast<float*>(ws + L.p_v);
+  p.p_s = reinterpret_cast<float*>(ws + L.p_s);
+  p.mu = reinterpret_cast<float*>(ws + L.mu);
+  p.vs_mask = reinterpret_cast<uint32_t*>(ws + L.vs_mask);
+  p.v_idx = reinterpret_cast<int32_t*>(ws + L.v_idx);
+  p.s_idx = reinterpret_cast<int32_t*>(ws + L.s_idx);
+  p.nv = reinterpret_cast<int32_t*>(ws + L.nv);
+  p.ns = reinterpret_cast<int32_t*>(ws + L.ns);
+  p.pe_mask = reinterpret_cast<uint32_t*>(ws + L.pe_mask);
+  p.pe_count = reinterpret_cast<int64_t*>(ws + L.pe_count);
+  p.pe_cut = reinterpret_cast<float*>(ws + L.pe_cut);
+  return p;
+}
+
+static crisp_status make_shape(const crisp_cfg* c, Shape* s) {
+  if (c == nullptr) return CRISP_ERR_INVALID_ARG;
+  if (c->reserved != 0) return CRISP_ERR_INVALID_ARG;
+  if (c->dtype != CRISP_BF16 && c->dtype != CRISP_FP32) return CRISP_ERR_DTYPE;
+  if (c->d != kHeadDim) return CRISP_ERR_SHAPE;
+  if (c->n < 512 || c->n % kBlock != 0 || c->n > (1 << 20)) return CRISP_ERR_SHAPE;
+  if (c->h_q <= 0 || c->h_kv <= 0 || c->h_q % c->h_kv != 0 || c->h_q / c->h_kv > 16 || c->h_q > 1024)
+    return CRISP_ERR_SHAPE;
+  if (c->block != kBlock || c->last_q != kProxyRows || c->w_sink != kBlock || c->w_local != kBlock)
+    return CRISP_ERR_UNSUPPORTED;
+  if (!isfinite(c->tau_proxy) || !isfinite(c->alpha) || c->alpha < 0.f) return CRISP_ERR_INVALID_ARG;
+  if (!(c->gamma > 0.f && c->gamma <= 1.f)) return CRISP_ERR_INVALID_ARG;
+  if (!isfinite(c->sm_scale)) return CRISP_ERR_INVALID_ARG;
+  if (c->force_route < -1 || c->force_route > 1) return CRISP_ERR_INVALID_ARG;
+  s->n = c->n;
+  s->h_q = c->h_q;
+  s->h_kv = c->h_kv;
+  s->d = c->d;
+  s->group = c->h_q / c->h_kv;
+  s->nb = c->n / kBlock;
+  s->words = (s->nb + 31) / 32;
+  s->n_chunks = (s->nb + kChunkTiles - 1) / kChunkTiles;
+  s->last_q = c->last_q;
+  s->tri = (long long)s->nb * (s->nb + 1) / 2;
+  s->fp32 = c->dtype == CRISP_FP32;
+  s->sm_scale = c->sm_scale > 0.f ? c->sm_scale : 1.f / sqrtf((float)c->d);
+  s->scale_log2 = s->sm_scale * 1.4426950408889634f;
+  s->tau = c->tau_proxy;
+  s->alpha = c->alpha;
+  s->gamma = c->gamma;
+  s->force_route = c->force_route;
+  return CRISP_OK;
+}
+
+static crisp_status check_tensor(const void* p) {
+  if (p == nullptr) return CRISP_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(p) % 16 != 0) return CRISP_ERR_ALIGN;
+  return CRISP_OK;
+}
+
+static crisp_status check_ws(const crisp_cfg* c, const WsLayout& L) {
+  if (c->workspace == nullptr) return CRISP_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(c->workspace) % 256 != 0) return CRISP_ERR_ALIGN;
+  if (c->workspace_bytes < L.total) return CRISP_ERR_WORKSPACE;
+  return CRISP_OK;
+}
+
+static crisp_status check_index(const crisp_index* ix, bool full) {
+  if (ix == nullptr) return CRISP_ERR_INVALID_ARG;
+  const void* need[] = {ix->route, ix->vs_mask, ix->pe_mask};
+  for (const void* p : need)
+    if (p == nullptr) return CRISP_ERR_INVALID_ARG;
+  if (full) {
+    const void* all[] = {ix->c_struct, ix->p_v, ix->p_s, ix->mu, ix->v_idx, ix->s_idx,
+                         ix->nv, ix->ns, ix->pe_count, ix->pe_cut};
+    for (const void* p : all)
+      if (p == nullptr) return CRISP_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(ix->pe_count) % 8 != 0) return CRISP_ERR_ALIGN;
+  }
+  const void* al[] = {ix->route, ix->vs_mask, ix->pe_mask, ix->c_struct, ix->p_v, ix->p_s, ix->mu,
+                      ix->v_idx, ix->s_idx, ix->nv, ix->ns, ix->pe_cut};
+  for (const void* p : al)
+    if (p != nullptr && reinterpret_cast<uintptr_t>(p) % 4 != 0) return CRISP_ERR_ALIGN;
+  return CRISP_OK;
+}
+
+static IndexPtrs from_abi(const crisp_index* ix) {
+  IndexPtrs p;
+  p.route = ix->route;
+  p.c_struct = ix->c_struct;
+  p.p_v = ix->p_v;
+  p.p_s = ix->p_s;
+  p.mu = ix->mu;
+  p.vs_mask = ix->vs_mask;
+  p.v_idx = ix->v_idx;
+  p.s_idx = ix->s_idx;
+  p.nv = ix->nv;
+  p.ns = ix->ns;
+  p.pe_mask = ix->pe_mask;
+  p.pe_count = ix->pe_count;
+  p.pe_cut = ix->pe_cut;
+  return p;
+}
+
+#define CRISP_TRY(expr)                         \
+  do {                                          \
+    if ((expr) != cudaSuccess) {                \
+      (void)cudaGetLastError();                 \
+      return CRISP_ERR_CUDA;                    \
+    }                                           \
+  } while (0)
+
+// Algorithm 2 (proxy map, finalisation, route) and Algorithm 3's selection;
+// Algorithm 4 too when `with_pe`.
+static crisp_status run_index(const void* q, const void* k, const Shape& s, char* ws, const WsLayout& L,
+                              const IndexPtrs& ix, bool with_pe, cudaStream_t st) {
+  CRISP_TRY(cudaMemsetAsync(ws + L.kv_pe, 0, (size_t)s.h_kv * 4, st));
+  CRISP_TRY(launch_proxy_simt(q, k, s, ws, L, st));
+  CRISP_TRY(launch_finalize(s, ws, L, ix, st));
+  CRISP_TRY(launch_vs_select(s, ws, L, ix, st));
+  if (with_pe) CRISP_TRY(launch_pe(q, k, s, ws, L, ix, st));
+  return CRISP_OK;
+}
+
+static crisp_status run_attention(const void* q, const void* k, const void* v, void* out, const Shape& s,
+                                  char* ws, const WsLayout& L, const int32_t* route, const uint32_t* vs_mask,
+                                  const uint32_t* pe_mask, bool dense, cudaStream_t st) {
+  int32_t* status = reinterpret_cast<int32_t*>(ws + L.status);
+  if (!s.fp32 && use_tensor_cores())
+    CRISP_TRY(launch_attn_tc(q, k, v, out, s, route, vs_mask, pe_mask, dense, status, st));
+  else
+    CRISP_TRY(launch_attn_simt(q, k, v, out, s, route, vs_mask, pe_mask, dense, status, st));
+  return CRISP_OK;
+}
+
+// Validate a call that reads q, k (and v, out when given) and uses the workspace.
+static crisp_status prepare(const crisp_cfg* cfg, const void* q, const void* k, const void* v, const void* out,
+                            bool need_vo, Shape* s, WsLayout* L) {
+  crisp_status r = make_shape(cfg, s);
+  if (r != CRISP_OK) return r;
+  if ((r = check_tensor(q)) != CRISP_OK) return r;
+  if ((r = check_tensor(k)) != CRISP_OK) return r;
+  if (need_vo) {
+    if ((r = check_tensor(v)) != CRISP_OK) return r;
+    if ((r = check_tensor(out)) != CRISP_OK) return r;
+  }
+  *L = ws_layout(*s);
+  return check_ws(cfg, *L);
+}
+
+}  // namespace crisp
+
+using namespace crisp;
+
+extern "C" {
+
+crisp_status crisp_cfg_init(crisp_cfg* cfg, int32_t n, int32_t h_q, int32_t h_kv, int32_t d, int32_t dtype) {
+  if (cfg == nullptr) return CRISP_ERR_INVALID_ARG;
+  memset(cfg, 0, sizeof(*cfg));
+  cfg->n = n;
+  cfg->h_q = h_q;
+  cfg->h_kv = h_kv;
+  cfg->d = d;
+  cfg->dtype = dtype;
+  cfg->block = kBlock;
+  cfg->last_q = kProxyRows;
+  cfg->w_sink = kBlock;
+  cfg->w_local = kBlock;
+  cfg->tau_proxy = 0.10f;
+  cfg->alpha = 1.0f;
+  cfg->gamma = 0.95f;
+  cfg->sm_scale = 0.f;
+  cfg->force_route = CRISP_ROUTE_AUTO;
+  return CRISP_OK;
+}
+
+crisp_status crisp_workspace_size(const crisp_cfg* cfg, size_t* bytes) {
+  Shape s;
+  crisp_status r = make_shape(cfg, &s);
+  if (r != CRISP_OK) return r;
+  if (bytes == nullptr) return CRISP_ERR_INVALID_ARG;
+  *bytes = ws_layout(s).total;
+  return CRISP_OK;
+}
+
+crisp_status crisp_index_dims(const crisp_cfg* cfg, int32_t* n_blocks, int32_t* words) {
+  Shape s;
+  crisp_status r = make_shape(cfg, &s);
+  if (r != CRISP_OK) return r;
+  if (n_blocks == nullptr || words == nullptr) return CRISP_ERR_INVALID_ARG;
+  *n_blocks = s.nb;
+  *words = s.words;
+  return CRISP_OK;
+}
+
+crisp_status crisp_route(const void* q, const void* k, const crisp_cfg* cfg, int32_t* route, float* c_struct,
+                         void* stream) {
+  Shape s;
+  WsLayout L;
+  crisp_status r = prepare(cfg, q, k, nullptr, nullptr, false, &s, &L);
+  if (r != CRISP_OK) return r;
+  if (route == nullptr || c_struct == nullptr) return CRISP_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(cfg->workspace);
+  CRISP_TRY(cudaMemsetAsync(ws + L.status, 0, 32, st));
+  IndexPtrs ix = internal_index(ws, L);
+  r = run_index(q, k, s, ws, L, ix, false, st);
+  if (r != CRISP_OK) return r;
+  CRISP_TRY(cudaMemcpyAsync(route, ix.route, (size_t)s.h_q * 4, cudaMemcpyDeviceToDevice, st));
+  CRISP_TRY(cudaMemcpyAsync(c_struct, ix.c_struct, (size_t)s.h_q * 4, cudaMemcpyDeviceToDevice, st));
+  return CRISP_OK;
+}
+
+crisp_status crisp_select(const void* q, const void* k, const crisp_cfg* cfg, const crisp_index* index,
+                          void* stream) {
+  Shape s;
+  WsLayout L;
+  crisp_status r = prepare(cfg, q, k, nullptr, nullptr, false, &s, &L);
+  if (r != CRISP_OK) return r;
+  if ((r = check_index(index, true)) != CRISP_OK) return r;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(cfg->workspace);
+  CRISP_TRY(cudaMemsetAsync(ws + L.status, 0, 32, st));
+  return run_index(q, k, s, ws, L, from_abi(index), true, st);
+}
+
+crisp_status crisp_attend(const void* q, const void* k, const void* v, void* out, const crisp_cfg* cfg,
+                          const crisp_index* index, void* stream) {
+  Shape s;
+  WsLayout L;
+  crisp_status r = prepare(cfg, q, k, v, out, true, &s, &L);
+  if (r != CRISP_OK) return r;
+  if ((r = check_index(index, false)) != CRISP_OK) return r;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(cfg->workspace);
+  CRISP_TRY(cudaMemsetAsync(ws + L.status, 0, 32, st));
+  return run_attention(q, k, v, out, s, ws, L, index->route, index->vs_mask, index->pe_mask, false, st);
+}
+
+crisp_status crisp_prefill(const void* q, const void* k, const void* v, void* out, const crisp_cfg* cfg,
+                           void* stream) {
+  Shape s;
+  WsLayout L;
+  crisp_status r = prepare(cfg, q, k, v, out, true, &s, &L);
+  if (r != CRISP_OK) return r;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(cfg->workspace);
+  CRISP_TRY(cudaMemsetAsync(ws + L.status, 0, 32, st));
+  IndexPtrs ix = internal_index(ws, L);
+  r = run_index(q, k, s, ws, L, ix, true, st);
+  if (r != CRISP_OK) return r;
+  return run_attention(q, k, v, out, s, ws, L, ix.route, ix.vs_mask, ix.pe_mask, false, st);
+}
+
+crisp_status crisp_dense_attention(const void* q, const void* k, const void* v, void* out, const crisp_cfg* cfg,
+                                   void* stream) {
+  Shape s;
+  WsLayout L;
+  crisp_status r = prepare(cfg, q, k, v, out, true, &s, &L);
+  if (r != CRISP_OK) return r;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(cfg->workspace);
+  CRISP_TRY(cudaMemsetAsync(ws + L.status, 0, 32, st));
+  return run_attention(q, k, v, out, s, ws, L, nullptr, nullptr, nullptr, true, st);
+}
+
+crisp_status crisp_device_status(const crisp_cfg* cfg, void* stream, int32_t* device_status) {
+  Shape s;
+  crisp_status r = make_shape(cfg, &s);
+  if (r != CRISP_OK) return r;
+  if (device_status == nullptr) return CRISP_ERR_INVALID_ARG;
+  WsLayout L = ws_layout(s);
+  if ((r = check_ws(cfg, L)) != CRISP_OK) return r;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(cfg->workspace);
+  int32_t word[2] = {0, 0};
+  CRISP_TRY(cudaStreamSynchronize(st));
+  CRISP_TRY(cudaMemcpy(word, ws + L.status, sizeof(word), cudaMemcpyDeviceToHost));
+  CRISP_TRY(cudaMemset(ws + L.status, 0, 32));
+  *device_status = word[0];
+  return CRISP_OK;
+}
+
+const char* crisp_status_string(crisp_status status) {
+  switch (status) {
+    case CRISP_OK: return "ok";
+    case CRISP_ERR_INVALID_ARG: return "invalid argument";
+    case CRISP_ERR_SHAPE: return "unsupported shape";
+    case CRISP_ERR_DTYPE: return "unsupported element type";
+    case CRISP_ERR_ALIGN: return "misaligned pointer";
+    case CRISP_ERR_WORKSPACE: return "workspace missing or too small";
+    case CRISP_ERR_UNSUPPORTED: return "unsupported parameter value";
+    case CRISP_ERR_CUDA: return "CUDA runtime error";
+    case CRISP_ERR_CAPACITY: return "device buffer capacity exceeded";
+    case CRISP_ERR_TIMEOUT: return "device wait timed out";
+    case CRISP_ERR_NONFINITE: return "non-finite proxy statistic";
+  }
+  return "unknown status";
+}
+
+int32_t crisp_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,441 @@
+// Pooled estimation (CRISP summary page, Algorithm 4, "GlobalAdaptive"):
+// block-mean pooling of Q and K, A-bar = softmax(Q-bar K-bar^T * sm_scale)
+// over c <= r, normalisation of the flattened causal map by its total (N_b,
+// one per row), and the gamma-cumulative cut: keep the largest entries
+// (ties by ascending flat index r*N_b + c) until their mass reaches gamma.
+// The diagonal block is always kept.
+//
+// The cut is found without sorting: a three-level radix select over the
+// fp32 bit patterns of the (positive) entries, with per-bucket counts and
+// float64 mass. Only heads routed PE do any work; the rest exit at once.
+#include <cuda_bf16.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace crisp {
+namespace {
+
+struct PeArgs {
+  int n, nb, words, group, h_q, h_kv;
+  long long tri;
+  float scale_log2;
+  float gamma;
+  const int32_t* route;
+  const int32_t* kv_pe;
+  float* qbar;
+  float* kbar;
+  float* tri_buf;
+  PeHist* hist;
+  PeState* state;
+  uint32_t* tie_rows;
+  uint32_t* pe_mask;
+  int64_t* pe_count;
+  float* pe_cut;
+  int32_t* status;
+};
+
+__device__ __forceinline__ long long tri_off(int r) { return (long long)r * (r + 1) / 2; }
+
+// Block mean of 128 rows of x[head] -> out[head][b][:] (fp32). One CTA per (block, head).
+template <typename T>
+__global__ void __launch_bounds__(128) pool_kernel(const T* __restrict__ x, float* __restrict__ out, int n, int nb,
+                                                   const int32_t* __restrict__ flag, int flag_div) {
+  const int b = blockIdx.x, head = blockIdx.y;
+  if (flag[head / flag_div] == 0) return;   // route check (query heads) or group check (KV heads)
+  __shared__ float red[8][kHeadDim];
+  const int tid = threadIdx.x, rg = tid >> 4, c8 = (tid & 15) * 8;
+  float acc[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+  const T* base = x + ((size_t)head * n + (size_t)b * kBlock) * kHeadDim;
+  for (int row = rg; row < kBlock; row += 8) {
+    const T* p = base + (size_t)row * kHeadDim + c8;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[j] += dev::to_f32(p[j]);
+  }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) red[rg][c8 + j] = acc[j];
+  __syncthreads();
+  float s = 0.f;
+#pragma unroll
+  for (int g = 0; g < 8; ++g) s += red[g][tid];
+  out[((size_t)head * nb + b) * kHeadDim + tid] = s * (1.f / kBlock);
+}
+
+// Pooled logits (log2 domain) of 16 query blocks against all key blocks c <= r.
+__global__ void __launch_bounds__(256) pe_logits_kernel(PeArgs a) {
+  const int h = blockIdx.y;
+  if (a.route[h] != 1) return;
+  const int g = h / a.group;
+  const int r0 = blockIdx.x * 16;
+  __shared__ float qs[16][kHeadDim + 1];
+  __shared__ float ksm[64][kHeadDim + 1];
+  const int tid = threadIdx.x;
+  for (int e = tid; e < 16 * kHeadDim; e += 256) {
+    const int rr = e >> 7, dd = e & 127;
+    qs[rr][dd] = (r0 + rr < a.nb) ? a.qbar[((size_t)h * a.nb + r0 + rr) * kHeadDim + dd] * a.scale_log2 : 0.f;
+  }
+  const int ri = tid >> 4, cj = tid & 15;
+  const int r = r0 + ri;
+  const int rmax = min(r0 + 15, a.nb - 1);
+  for (int c0 = 0; c0 <= rmax; c0 += 64) {
+    __syncthreads();
+    for (int e = tid; e < 64 * kHeadDim; e += 256) {
+      const int cc = e >> 7, dd = e & 127;
+      ksm[cc][dd] = (c0 + cc < a.nb) ? a.kbar[((size_t)g * a.nb + c0 + cc) * kHeadDim + dd] : 0.f;
+    }
+    __syncthreads();
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int dd = 0; dd < kHeadDim; ++dd) {
+      const float qv = qs[ri][dd];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) acc[u] = fmaf(qv, ksm[cj + 16 * u][dd], acc[u]);
+    }
+    if (r < a.nb) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int c = c0 + cj + 16 * u;
+        if (c <= r) a.tri_buf[(size_t)h * a.tri + tri_off(r) + c] = acc[u];
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void hist_flush(PeHist* hist, uint32_t bucket, unsigned long long cnt, double mass) {
+  if (cnt == 0) return;
+  atomicAdd(&hist->count[bucket], cnt);
+  atomicAdd(&hist->mass[bucket], mass);
+}
+
+__device__ float block_reduce_max(float v, float* sh) {
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  if ((threadIdx.x & 31) == 0) sh[threadIdx.x >> 5] = v;
+  __syncthreads();
+  float r = -INFINITY;
+  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) r = fmaxf(r, sh[w]);
+  __syncthreads();
+  return r;
+}
+__device__ float block_reduce_sum(float v, float* sh) {
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if ((threadIdx.x & 31) == 0) sh[threadIdx.x >> 5] = v;
+  __syncthreads();
+  float r = 0.f;
+  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) r += sh[w];
+  __syncthreads();
+  return r;
+}
+
+// Row softmax of the pooled logits, divided by N_b (the flattened map's total),
+// written in place; level-0 histogram (bits 31..20) with float64 mass.
+__global__ void __launch_bounds__(256) pe_softmax_kernel(PeArgs a) {
+  const int h = blockIdx.y, r = blockIdx.x;
+  if (a.route[h] != 1) return;
+  __shared__ float sh[32];
+  float* row = a.tri_buf + (size_t)h * a.tri + tri_off(r);
+  float m = -INFINITY;
+  for (int c = threadIdx.x; c <= r; c += blockDim.x) m = fmaxf(m, row[c]);
+  m = block_reduce_max(m, sh);
+  float s = 0.f;
+  for (int c = threadIdx.x; c <= r; c += blockDim.x) s += dev::ex2(row[c] - m);
+  s = block_reduce_sum(s, sh);
+  const float inv = 1.f / (s * (float)a.nb);
+  PeHist* hist = a.hist + h;
+  uint32_t cur = 0xffffffffu;
+  unsigned long long cnt = 0;
+  double mass = 0.0;
+  for (int c = threadIdx.x; c <= r; c += blockDim.x) {
+    const float v = dev::ex2(row[c] - m) * inv;
+    row[c] = v;
+    const uint32_t bucket = __float_as_uint(v) >> 20;
+    if (bucket != cur) {
+      if (cur != 0xffffffffu) hist_flush(hist, cur, cnt, mass);
+      cur = bucket;
+      cnt = 0;
+      mass = 0.0;
+    }
+    ++cnt;
+    mass += (double)v;
+  }
+  if (cur != 0xffffffffu) hist_flush(hist, cur, cnt, mass);
+}
+
+// Histogram of the entries whose key matches the prefix found so far
+// (level 1: bits 19..8 under the 12-bit prefix; level 2: bits 7..0 under the 24-bit prefix).
+__global__ void __launch_bounds__(256) pe_hist_kernel(PeArgs a, int level) {
+  const int h = blockIdx.y;
+  if (a.route[h] != 1) return;
+  const PeState* st = a.state + h;
+  if (st->all) return;
+  const uint32_t prefix = st->prefix;
+  const int shift_p = level == 1 ? 20 : 8;
+  const int shift_b = level == 1 ? 8 : 0;
+  const uint32_t bmask = level == 1 ? 0xFFFu : 0xFFu;
+  const float* tri = a.tri_buf + (size_t)h * a.tri;
+  PeHist* hist = a.hist + h;
+  for (long long p = (long long)blockIdx.x * blockDim.x + threadIdx.x; p < a.tri;
+       p += (long long)gridDim.x * blockDim.x) {
+    const float v = tri[p];
+    const uint32_t key = __float_as_uint(v);
+    if ((key >> shift_p) == prefix) {
+      const uint32_t b = (key >> shift_b) & bmask;
+      atomicAdd(&hist->count[b], 1ull);
+      atomicAdd(&hist->mass[b], (double)v);
+    }
+  }
+}
+
+// Walk the buckets of the current level from the largest key down, carrying
+// the mass above; pick the bucket where the cumulative mass reaches gamma.
+// One CTA (1024 threads) per head. Clears the histogram for the next level.
+__global__ void __launch_bounds__(1024) pe_find_kernel(PeArgs a, int level) {
+  const int h = blockIdx.x;
+  if (a.route[h] != 1) return;
+  PeState* st = a.state + h;
+  PeHist* hist = a.hist + h;
+  const int nbk = level == 2 ? kHistL2 : kHistL0;
+  const int per = (nbk + 1023) / 1024;
+  __shared__ double tsum[1024];
+  __shared__ int s_found;
+  __shared__ double s_above_new;
+  __shared__ int s_bucket;
+  const int tid = threadIdx.x;
+  if (tid == 0) {
+    if (level == 0) {
+      st->s_above = 0.0;
+      st->prefix = 0;
+      st->all = a.gamma >= 1.f ? 1u : 0u;
+    }
+    s_found = 0;
+  }
+  __syncthreads();
+  const bool all = st->all != 0;
+  // thread tid owns descending buckets [nbk-1 - tid*per, ... - per + 1]
+  double my = 0.0;
+  for (int u = 0; u < per; ++u) {
+    const int b = nbk - 1 - (tid * per + u);
+    if (b >= 0) my += hist->mass[b];
+  }
+  tsum[tid] = my;
+  __syncthreads();
+  // inclusive scan over threads (descending bucket order)
+  for (int off = 1; off < 1024; off <<= 1) {
+    const double v = tid >= off ? tsum[tid - off] : 0.0;
+    __syncthreads();
+    tsum[tid] += v;
+    __syncthreads();
+  }
+  if (level == 0 && tid == 0) st->total = tsum[1023];
+  __syncthreads();
+  const double base = st->s_above;
+  const double gamma = (double)a.gamma;
+  if (!all) {
+    const double before = base + (tid > 0 ? tsum[tid - 1] : 0.0);
+    const double after = base + tsum[tid];
+    if (before < gamma && after >= gamma) {
+      double acc = before;
+      int last_b = -1;
+      double last_above = 0.0;
+      for (int u = 0; u < per; ++u) {
+        const int b = nbk - 1 - (tid * per + u);
+        if (b < 0) break;
+        if (hist->count[b] == 0) continue;
+        last_b = b;
+        last_above = acc;
+        const double nxt = acc + hist->mass[b];
+        if (nxt >= gamma) break;
+        acc = nxt;
+      }
+      if (last_b >= 0) {   // the crossing bucket (or, after rounding, the lowest one of this thread)
+        s_bucket = last_b;
+        s_above_new = last_above;
+        s_found = 1;
+      }
+    }
+  }
+  __syncthreads();
+  if (!all && !s_found && level > 0 && tid == 0) {
+    // Summation order can leave the children of the crossing bucket a hair
+    // short of gamma; the crossing then lies in the lowest non-empty child.
+    for (int b = 0; b < nbk; ++b) {
+      if (hist->count[b] > 0) {
+        s_bucket = b;
+        s_above_new = base + (tsum[1023] - hist->mass[b]);
+        s_found = 1;
+        break;
+      }
+    }
+  }
+  __syncthreads();
+  if (tid == 0 && !all) {
+    if (!s_found) {
+      st->all = 1u;   // the cumulative mass never reaches gamma: keep everything
+    } else {
+      const int bits = level == 2 ? 8 : 12;
+      st->s_above = s_above_new;
+      st->prefix = (st->prefix << bits) | (uint32_t)s_bucket;
+      if (level == 2) {
+        const uint32_t key = st->prefix;
+        const double v = (double)__uint_as_float(key);
+        const unsigned long long nt = hist->count[s_bucket];
+        double need = (gamma - st->s_above) / v;
+        unsigned long long t = need <= 1.0 ? 1ull : (unsigned long long)ceil(need);
+        while (t > 1 && st->s_above + (double)(t - 1) * v >= gamma) --t;
+        while (t < nt && st->s_above + (double)t * v < gamma) ++t;
+        if (t > nt) t = nt;
+        st->cut_key = key;
+        st->n_ties = nt;
+        st->t_keep = t;
+      }
+    }
+  }
+  __syncthreads();
+  for (int b = tid; b < kHistL0; b += 1024) {
+    hist->count[b] = 0;
+    hist->mass[b] = 0.0;
+  }
+}
+
+// Ties needed in part only: count entries equal to the cut value per row.
+__global__ void __launch_bounds__(256) pe_tie_count_kernel(PeArgs a) {
+  const int h = blockIdx.y, r = blockIdx.x;
+  if (a.route[h] != 1) return;
+  const PeState* st = a.state + h;
+  if (st->all || st->t_keep >= st->n_ties) return;
+  __shared__ float sh[32];
+  const float* row = a.tri_buf + (size_t)h * a.tri + tri_off(r);
+  float cnt = 0.f;
+  for (int c = threadIdx.x; c <= r; c += blockDim.x) cnt += (__float_as_uint(row[c]) == st->cut_key) ? 1.f : 0.f;
+  cnt = block_reduce_sum(cnt, sh);
+  if (threadIdx.x == 0) a.tie_rows[(size_t)h * a.nb + r] = (uint32_t)cnt;
+}
+
+__global__ void __launch_bounds__(32) pe_tie_scan_kernel(PeArgs a) {
+  const int h = blockIdx.x;
+  if (a.route[h] != 1) return;
+  const PeState* st = a.state + h;
+  if (st->all || st->t_keep >= st->n_ties) return;
+  if (threadIdx.x != 0) return;
+  uint32_t acc = 0;
+  for (int r = 0; r < a.nb; ++r) {
+    const uint32_t v = a.tie_rows[(size_t)h * a.nb + r];
+    a.tie_rows[(size_t)h * a.nb + r] = acc;
+    acc += v;
+  }
+}
+
+// Write the PE mask row by row: keep (r, c), c <= r, when its value is above
+// the cut, or equal to it and among the first t_keep ties in flat order, or
+// c == r; or everything when the cut keeps all.
+__global__ void __launch_bounds__(256) pe_mask_kernel(PeArgs a) {
+  const int h = blockIdx.y, r = blockIdx.x;
+  if (a.route[h] != 1) return;
+  const PeState* st = a.state + h;
+  __shared__ int warp_sums[9];
+  __shared__ float shr[32];
+  const bool all = st->all != 0;
+  const uint32_t cut = st->cut_key;
+  const bool partial_ties = !all && st->t_keep < st->n_ties;
+  const unsigned long long t_keep = st->t_keep;
+  unsigned long long tie_base = partial_ties ? a.tie_rows[(size_t)h * a.nb + r] : 0ull;
+  const float* row = a.tri_buf + (size_t)h * a.tri + tri_off(r);
+  uint32_t* mrow = a.pe_mask + ((size_t)h * a.nb + r) * a.words;
+  float kept = 0.f;
+  for (int c0 = 0; c0 < a.words * 32; c0 += blockDim.x) {
+    const int c = c0 + threadIdx.x;
+    int keep = 0, tie = 0;
+    if (c <= r) {
+      const uint32_t key = __float_as_uint(row[c]);
+      tie = (!all && key == cut) ? 1 : 0;
+      keep = all || c == r || key > cut || (tie && !partial_ties);
+    }
+    if (partial_ties) {
+      // rank of this tie among the ties of the head in flat order
+      const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+      const unsigned bal = __ballot_sync(0xffffffffu, tie);
+      if (lane == 0) warp_sums[wid] = __popc(bal);
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        int acc = 0;
+        for (int w = 0; w < 8; ++w) {
+          const int v = warp_sums[w];
+          warp_sums[w] = acc;
+          acc += v;
+        }
+        warp_sums[8] = acc;
+      }
+      __syncthreads();
+      const unsigned long long rank = tie_base + warp_sums[wid] + __popc(bal & ((1u << lane) - 1u));
+      if (tie && rank < t_keep) keep = 1;
+      tie_base += warp_sums[8];
+      __syncthreads();
+    }
+    const unsigned bal = __ballot_sync(0xffffffffu, keep);
+    if ((threadIdx.x & 31) == 0 && (c >> 5) < a.words) mrow[c >> 5] = bal;
+    kept += keep ? 1.f : 0.f;
+  }
+  kept = block_reduce_sum(kept, shr);
+  if (threadIdx.x == 0) {
+    atomicAdd(reinterpret_cast<unsigned long long*>(a.pe_count + h), (unsigned long long)kept);
+    if (r == 0) a.pe_cut[h] = all ? 0.f : __uint_as_float(cut);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_pe(const void* q, const void* k, const Shape& s, char* ws, const WsLayout& L,
+                      const IndexPtrs& ix, cudaStream_t st) {
+  PeArgs a;
+  a.n = s.n;
+  a.nb = s.nb;
+  a.words = s.words;
+  a.group = s.group;
+  a.h_q = s.h_q;
+  a.h_kv = s.h_kv;
+  a.tri = s.tri;
+  a.scale_log2 = s.scale_log2;
+  a.gamma = s.gamma;
+  a.route = ix.route;
+  a.kv_pe = reinterpret_cast<const int32_t*>(ws + L.kv_pe);
+  a.qbar = reinterpret_cast<float*>(ws + L.qbar);
+  a.kbar = reinterpret_cast<float*>(ws + L.kbar);
+  a.tri_buf = reinterpret_cast<float*>(ws + L.tri);
+  a.hist = reinterpret_cast<PeHist*>(ws + L.hist);
+  a.state = reinterpret_cast<PeState*>(ws + L.pe_state);
+  a.tie_rows = reinterpret_cast<uint32_t*>(ws + L.tie_rows);
+  a.pe_mask = ix.pe_mask;
+  a.pe_count = ix.pe_count;
+  a.pe_cut = ix.pe_cut;
+  a.status = reinterpret_cast<int32_t*>(ws + L.status);
+
+  cudaError_t e = cudaMemsetAsync(a.hist, 0, sizeof(PeHist) * s.h_q, st);
+  if (e != cudaSuccess) return e;
+  // the query-head pooling is gated by the route; the key pooling by kv_pe
+  // (route values 1 = PE are used directly as the flag).
+  if (s.fp32) {
+    pool_kernel<float><<<dim3(s.nb, s.h_q), 128, 0, st>>>(static_cast<const float*>(q), a.qbar, s.n, s.nb,
+                                                          ix.route, 1);
+    pool_kernel<float><<<dim3(s.nb, s.h_kv), 128, 0, st>>>(static_cast<const float*>(k), a.kbar, s.n, s.nb,
+                                                           a.kv_pe, 1);
+  } else {
+    pool_kernel<__nv_bfloat16><<<dim3(s.nb, s.h_q), 128, 0, st>>>(static_cast<const __nv_bfloat16*>(q), a.qbar,
+                                                                  s.n, s.nb, ix.route, 1);
+    pool_kernel<__nv_bfloat16><<<dim3(s.nb, s.h_kv), 128, 0, st>>>(static_cast<const __nv_bfloat16*>(k), a.kbar,
+                                                                   s.n, s.nb, a.kv_pe, 1);
+  }
+  pe_logits_kernel<<<dim3((s.nb + 15) / 16, s.h_q), 256, 0, st>>>(a);
+  pe_softmax_kernel<<<dim3(s.nb, s.h_q), 256, 0, st>>>(a);
+  pe_find_kernel<<<s.h_q, 1024, 0, st>>>(a, 0);
+  const int hist_ctas = (int)std::min<long long>(1184, (s.tri + 255) / 256);
+  pe_hist_kernel<<<dim3(hist_ctas, s.h_q), 256, 0, st>>>(a, 1);
+  pe_find_kernel<<<s.h_q, 1024, 0, st>>>(a, 1);
+  pe_hist_kernel<<<dim3(hist_ctas, s.h_q), 256, 0, st>>>(a, 2);
+  pe_find_kernel<<<s.h_q, 1024, 0, st>>>(a, 2);
+  pe_tie_count_kernel<<<dim3(s.nb, s.h_q), 256, 0, st>>>(a);
+  pe_tie_scan_kernel<<<s.h_q, 32, 0, st>>>(a);
+  pe_mask_kernel<<<dim3(s.nb, s.h_q), 256, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace crisp

@@ -1,0 +1,140 @@
+"""The C-ABI library: it loads without a GPU, exports every function the
+header declares, its structs match ctypes' view, and host-side validation
+rejects bad arguments before anything is launched (no GPU needed)."""
+import ctypes
+import os
+import re
+import subprocess
+import tempfile
+
+import pytest
+
+import long_context_prefill_last_b200 as crisp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "crisp.h")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    from long_context_prefill_last_b200 import build
+    build.build()
+
+
+def header_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(crisp_[a-z_]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_function():
+    names = header_functions()
+    assert sorted(names) == sorted(crisp.SYMBOLS)
+    L = crisp.lib()
+    for n in names:
+        assert hasattr(L, n), n
+    out = subprocess.run(["nm", "-D", "--defined-only", crisp.library_path()], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\sT\s(crisp_\w+)", out))
+    assert set(names) <= exported
+
+
+def test_library_has_sm100a_code_and_no_undefined_cuda_driver_link():
+    out = subprocess.run(["ldd", crisp.library_path()], capture_output=True, text=True).stdout
+    assert "libcuda.so" not in out        # driver entry points are resolved at run time
+    assert "libcudart" not in out          # runtime is linked statically
+
+
+def test_struct_layout_matches_header():
+    src = r"""
+    #include <stdio.h>
+    #include <stddef.h>
+    #include "crisp.h"
+    int main(void) {
+      printf("%zu %zu %zu %zu %zu\n", sizeof(crisp_cfg), offsetof(crisp_cfg, tau_proxy),
+             offsetof(crisp_cfg, workspace), offsetof(crisp_cfg, workspace_bytes), sizeof(crisp_index));
+      return 0;
+    }"""
+    with tempfile.TemporaryDirectory() as d:
+        c = os.path.join(d, "t.c")
+        exe = os.path.join(d, "t")
+        open(c, "w").write(src)
+        subprocess.run(["gcc", "-I", os.path.dirname(HEADER), c, "-o", exe], check=True)
+        vals = [int(x) for x in subprocess.run([exe], capture_output=True, text=True).stdout.split()]
+    assert vals == [ctypes.sizeof(crisp._Cfg), crisp._Cfg.tau_proxy.offset, crisp._Cfg.workspace.offset,
+                    crisp._Cfg.workspace_bytes.offset, ctypes.sizeof(crisp._Index)]
+
+
+def test_cfg_init_defaults_match_python_config():
+    c = crisp._Cfg()
+    assert crisp.lib().crisp_cfg_init(ctypes.byref(c), 32768, 32, 8, 128, crisp.BF16) == 0
+    py = crisp.Config(n=32768, h_q=32, h_kv=8)._c()
+    for f, _ in crisp._Cfg._fields_:
+        assert getattr(c, f) == pytest.approx(getattr(py, f)), f
+
+
+def test_workspace_size_and_dims():
+    cfg = crisp.Config(n=524288, h_q=32, h_kv=8)
+    nb, w = crisp.index_dims(cfg)
+    assert (nb, w) == (4096, 128)
+    ws = crisp.workspace_size(cfg)
+    # dominated by the pooled PE triangle: h_q * N_b(N_b+1)/2 floats
+    assert 32 * 4096 * 4097 // 2 * 4 < ws < 2 * 2 ** 30
+
+
+@pytest.mark.parametrize("field,value,code", [
+    ("n", 1000, "CRISP_ERR_SHAPE"), ("n", 256, "CRISP_ERR_SHAPE"), ("n", 4095, "CRISP_ERR_SHAPE"),
+    ("d", 64, "CRISP_ERR_SHAPE"), ("h_kv", 3, "CRISP_ERR_SHAPE"), ("h_q", 0, "CRISP_ERR_SHAPE"),
+    ("dtype", 7, "CRISP_ERR_DTYPE"), ("block", 64, "CRISP_ERR_UNSUPPORTED"),
+    ("last_q", 128, "CRISP_ERR_UNSUPPORTED"), ("w_sink", 64, "CRISP_ERR_UNSUPPORTED"),
+    ("gamma", 0.0, "CRISP_ERR_INVALID_ARG"), ("gamma", 1.5, "CRISP_ERR_INVALID_ARG"),
+    ("alpha", -1.0, "CRISP_ERR_INVALID_ARG"), ("tau_proxy", float("nan"), "CRISP_ERR_INVALID_ARG"),
+    ("force_route", 2, "CRISP_ERR_INVALID_ARG"), ("reserved", 1, "CRISP_ERR_INVALID_ARG"),
+])
+def test_invalid_configs_are_rejected_on_the_host(field, value, code):
+    cfg = crisp.Config(n=4096, h_q=4, h_kv=2)
+    setattr(cfg, field, value)
+    with pytest.raises(crisp.CrispError) as e:
+        crisp.workspace_size(cfg)
+    assert crisp.STATUS_NAMES[e.value.code] == code
+
+
+class _FakeTensor:
+    def __init__(self, ptr, nbytes=0):
+        self.ptr, self.nbytes = ptr, nbytes
+
+    def data_ptr(self):
+        return self.ptr
+
+    def numel(self):
+        return self.nbytes
+
+    def element_size(self):
+        return 1
+
+
+def test_bad_pointers_and_workspace_fail_before_any_launch():
+    L = crisp.lib()
+    cfg = crisp.Config(n=4096, h_q=4, h_kv=2)
+    c = cfg._c()
+    # no workspace
+    assert L.crisp_prefill(0x10000, 0x20000, 0x30000, 0x40000, ctypes.byref(c), None) == 5
+    # null tensor
+    assert L.crisp_prefill(0, 0x20000, 0x30000, 0x40000, ctypes.byref(c), None) == 1
+    # misaligned tensor
+    assert L.crisp_dense_attention(0x10008, 0x20000, 0x30000, 0x40000, ctypes.byref(c), None) == 4
+    # workspace too small / misaligned
+    cfg.workspace = _FakeTensor(0x100000, 1024)
+    assert L.crisp_prefill(0x10000, 0x20000, 0x30000, 0x40000, ctypes.byref(cfg._c()), None) == 5
+    cfg.workspace = _FakeTensor(0x100010, 1 << 40)
+    assert L.crisp_route(0x10000, 0x20000, ctypes.byref(cfg._c()), 0x5000, 0x6000, None) == 4
+    # route outputs missing
+    cfg.workspace = _FakeTensor(0x100000, 1 << 40)
+    assert L.crisp_route(0x10000, 0x20000, ctypes.byref(cfg._c()), 0, 0x6000, None) == 1
+    # select without an index
+    assert L.crisp_select(0x10000, 0x20000, ctypes.byref(cfg._c()), None, None) == 1
+
+
+def test_status_strings():
+    assert crisp.status_string(0) == "ok"
+    assert "timed out" in crisp.status_string(9)
+    assert crisp.lib().crisp_version() >= 100

@@ -1,0 +1,270 @@
+"""CUDA path vs the CPU oracle, through the C ABI, on seeded synthetic layers.
+
+Routes and index sets must match bit for bit except documented flips
+(tests/parity.py); outputs on the same indices within 2e-2 (bf16) or 1e-4
+(fp32) max relative error. Small layers are checked on every row; the
+full-size layers on sampled query rows of every head.
+"""
+import os
+
+import numpy as np
+import pytest
+
+import crisp_synth as S
+from oracle import crisp_oracle as O
+import parity as P
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+import long_context_prefill_last_b200 as crisp  # noqa: E402
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    from long_context_prefill_last_b200 import build
+    build.build()
+    crisp.lib()
+
+
+def f32(x):
+    return float(np.float32(x))
+
+
+def oracle_cfg(cfg: crisp.Config) -> O.OracleCfg:
+    # the knobs exactly as the device sees them (float32)
+    return O.OracleCfg(tau_proxy=f32(cfg.tau_proxy), alpha=f32(cfg.alpha), gamma=f32(cfg.gamma),
+                       force_route=cfg.force_route)
+
+
+def device_layer(layer):
+    return tuple(t.cuda() for t in S.to_torch(layer))
+
+
+def make_cfg(layer, **kw):
+    c = layer.cfg
+    cfg = crisp.Config(n=c.n, h_q=c.h_q, h_kv=c.h_kv, d=c.d, dtype=crisp.FP32 if c.dtype == "fp32" else crisp.BF16,
+                       **kw)
+    cfg.allocate_workspace()
+    return cfg
+
+
+def gpu_select(q, k, cfg):
+    ix = crisp.IndexBuffers(cfg)
+    crisp.select(q, k, cfg, ix)
+    crisp.raise_on_device_status(cfg, where="select")
+    nb = cfg.n_blocks
+    host = {f: getattr(ix, f).cpu().numpy() for f in ("route", "c_struct", "p_v", "p_s", "mu", "nv", "ns",
+                                                       "pe_count", "pe_cut", "v_idx", "s_idx")}
+    host["sel_v"] = P.unpack_mask(ix.vs_mask[:, 0].cpu().numpy().view(np.uint32), nb)
+    host["sel_s"] = P.unpack_mask(ix.vs_mask[:, 1].cpu().numpy().view(np.uint32), nb)
+    host["pe"] = P.unpack_mask(ix.pe_mask.cpu().numpy().view(np.uint32), nb)
+    return host, ix
+
+
+def oracle_heads(layer, ocfg, heads=None):
+    G = layer.cfg.group
+    kcache = {}
+
+    def getk(g):
+        if g not in kcache:
+            kcache.clear()
+            kcache[g] = layer.as_f64("k", g)
+        return kcache[g]
+
+    out = {}
+    for h in (heads if heads is not None else range(layer.cfg.h_q)):
+        out[h] = O.head_index(layer.as_f64("q", h), getk(h // G), ocfg)
+    return out
+
+
+def check_index(host, oidx, cfg, rep):
+    for h, idx in oidx.items():
+        P.compare_route(h, float(host["c_struct"][h]), int(host["route"][h]), idx, f32(cfg.tau_proxy), rep)
+        P.compare_vs(h, host["sel_v"][h], host["sel_s"][h], idx, f32(cfg.alpha), rep)
+        # the compacted lists agree with the masks
+        nv, ns = int(host["nv"][h]), int(host["ns"][h])
+        assert (host["v_idx"][h][:nv] == np.nonzero(host["sel_v"][h])[0]).all()
+        assert (host["s_idx"][h][:ns] == np.nonzero(host["sel_s"][h])[0]).all()
+        if idx.route == O.PE and int(host["route"][h]) == O.PE:
+            P.compare_pe(h, host["pe"][h], idx, rep)
+            assert int(host["pe_count"][h]) == int(host["pe"][h][np.tril_indices(cfg.n_blocks)].sum())
+        # the block masses themselves (float32 device sums vs float64)
+        np.testing.assert_allclose(host["p_v"][h], idx.p_v, rtol=2e-3, atol=2e-6)
+        np.testing.assert_allclose(host["p_s"][h], idx.p_s, rtol=2e-3, atol=2e-6)
+
+
+def sample_rows(n, nb, full):
+    if full:
+        return np.arange(n)
+    tiles = sorted({0, 1, nb // 3, nb // 2, nb - 2, nb - 1})
+    rows = []
+    for t in tiles:
+        rows += [t * 128, t * 128 + 37, t * 128 + 64, t * 128 + 127]
+    return np.array(sorted(set(r for r in rows if r < n)))
+
+
+def check_outputs(layer, out, oidx, ocfg, rows, skip_heads=(), tol=None):
+    tol = tol if tol is not None else P.TOL[layer.cfg.dtype]
+    G = layer.cfg.group
+    o = out.float().cpu().numpy()
+    worst = 0.0
+    for h, idx in oidx.items():
+        if h in skip_heads:
+            continue
+        q, k, v = layer.as_f64("q", h), layer.as_f64("k", h // G), layer.as_f64("v", h // G)
+        ref = O.head_attention(q, k, v, idx, rows, ocfg)
+        err = P.output_error(o[h][rows], ref)
+        worst = max(worst, err)
+        assert err <= tol, f"head {h}: output error {err:.3g} > {tol}"
+    return worst
+
+
+def oracle_index_buffers(oidx, cfg):
+    """Device index buffers holding the ORACLE's route and masks (inputs for crisp_attend)."""
+    ix = crisp.IndexBuffers(cfg)
+    nb = cfg.n_blocks
+    h_q = cfg.h_q
+    route = np.zeros(h_q, np.int32)
+    vs = np.zeros((h_q, 2, cfg.words), np.uint32)
+    pe = np.zeros((h_q, nb, cfg.words), np.uint32)
+    for h, idx in oidx.items():
+        route[h] = idx.route
+        vs[h, 0] = P.pack_mask(idx.sel_v)
+        vs[h, 1] = P.pack_mask(idx.sel_s)
+        if idx.pe is not None:
+            pe[h] = P.pack_mask(idx.pe.mask)
+    ix.route.copy_(torch.from_numpy(route))
+    ix.vs_mask.copy_(torch.from_numpy(vs.view(np.int32)))
+    ix.pe_mask.copy_(torch.from_numpy(pe.view(np.int32)))
+    return ix
+
+
+# ----------------------------------------------------------------------------- small layers
+
+SMALL = {
+    "A-auto": (lambda: S.CONFIGS["A"], {}),
+    "A-forceVS": (lambda: S.CONFIGS["A"], {"force_route": 0}),
+    "B-4k": (lambda: S.scaled("B", n=4096, h_q=8, h_kv=2), {}),
+    "D-2k": (lambda: S.scaled("D", n=2048, h_q=14, h_kv=2), {}),
+    "B-512-min": (lambda: S.scaled("B", n=512, h_q=4, h_kv=1, planted_groups=[0]), {}),
+    "B-4224-33blocks": (lambda: S.scaled("B", n=4224, h_q=4, h_kv=2), {}),
+    "B-4k-alpha1.5": (lambda: S.scaled("B", n=4096, h_q=8, h_kv=2), {"alpha": 1.5}),
+    "B-4k-alpha0": (lambda: S.scaled("B", n=4096, h_q=8, h_kv=2), {"alpha": 0.0}),
+    "B-4k-gamma1": (lambda: S.scaled("B", n=4096, h_q=8, h_kv=2), {"gamma": 1.0}),
+    "B-4k-gamma0.5": (lambda: S.scaled("B", n=4096, h_q=8, h_kv=2), {"gamma": 0.5}),
+    "B-4k-forcePE": (lambda: S.scaled("B", n=4096, h_q=8, h_kv=2), {"force_route": 1}),
+    "B-4k-alphaHuge": (lambda: S.scaled("B", n=4096, h_q=8, h_kv=2), {"alpha": 1e30}),
+}
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_small_layer_parity(name):
+    make, knobs = SMALL[name]
+    layer = S.generate(make())
+    q, k, v = device_layer(layer)
+    cfg = make_cfg(layer, **knobs)
+    ocfg = oracle_cfg(cfg)
+    host, _ = gpu_select(q, k, cfg)
+    oidx = oracle_heads(layer, ocfg)
+    rep = P.Report()
+    check_index(host, oidx, cfg, rep)
+    rep.assert_ok()
+    # whole path; outputs compared where the indices agree exactly
+    out = torch.empty_like(q)
+    crisp.prefill(q, k, v, out, cfg)
+    crisp.raise_on_device_status(cfg, where="prefill")
+    rows = sample_rows(cfg.n, cfg.n_blocks, full=cfg.n <= 4224)
+    check_outputs(layer, out, oidx, ocfg, rows, skip_heads=rep.heads_with_flips())
+    # attention on the oracle's own indices, every head
+    ix = oracle_index_buffers(oidx, cfg)
+    out2 = torch.empty_like(q)
+    crisp.attend(q, k, v, out2, cfg, ix)
+    crisp.raise_on_device_status(cfg, where="attend")
+    check_outputs(layer, out2, oidx, ocfg, rows)
+
+
+@pytest.mark.parametrize("base,n,hq,hkv", [("A", 4096, 1, 1), ("B", 4096, 8, 2), ("D", 2048, 14, 2)])
+def test_dense_attention_parity(base, n, hq, hkv):
+    c = S.CONFIGS["A"] if base == "A" else S.scaled(base, n=n, h_q=hq, h_kv=hkv)
+    layer = S.generate(c)
+    q, k, v = device_layer(layer)
+    cfg = make_cfg(layer)
+    out = torch.empty_like(q)
+    crisp.dense_attention(q, k, v, out, cfg)
+    crisp.raise_on_device_status(cfg, where="dense")
+    o = out.float().cpu().numpy()
+    rows = np.arange(n) if n <= 4096 and hq <= 8 else sample_rows(n, n // 128, False)
+    tol = P.TOL[c.dtype]
+    for h in range(hq):
+        g = h // c.group
+        ref = O.dense_attention(layer.as_f64("q", h), layer.as_f64("k", g), layer.as_f64("v", g), rows,
+                                1 / np.sqrt(128))
+        assert P.output_error(o[h][rows], ref) <= tol
+
+
+def test_tensor_core_and_cuda_core_attention_agree():
+    layer = S.generate(S.scaled("B", n=4096, h_q=8, h_kv=2))
+    q, k, v = device_layer(layer)
+    cfg = make_cfg(layer)
+    ix = crisp.IndexBuffers(cfg)
+    crisp.select(q, k, cfg, ix)
+    outs = []
+    for force in ("0", "1"):
+        os.environ["CRISP_FORCE_SIMT"] = force
+        try:
+            o = torch.empty_like(q)
+            crisp.attend(q, k, v, o, cfg, ix)
+            crisp.raise_on_device_status(cfg)
+            outs.append(o.float())
+            o2 = torch.empty_like(q)
+            crisp.dense_attention(q, k, v, o2, cfg)
+            crisp.raise_on_device_status(cfg)
+            outs.append(o2.float())
+        finally:
+            os.environ.pop("CRISP_FORCE_SIMT", None)
+    for a, b in ((outs[0], outs[2]), (outs[1], outs[3])):
+        err = (a - b).abs().max().item() / b.abs().max().item()
+        assert err < 2e-2
+
+
+def test_repeat_calls_are_deterministic():
+    layer = S.generate(S.scaled("D", n=2048, h_q=14, h_kv=2))
+    q, k, v = device_layer(layer)
+    cfg = make_cfg(layer)
+    o1, o2 = torch.empty_like(q), torch.empty_like(q)
+    crisp.prefill(q, k, v, o1, cfg)
+    crisp.prefill(q, k, v, o2, cfg)
+    crisp.raise_on_device_status(cfg)
+    assert torch.equal(o1, o2)
+
+
+# ----------------------------------------------------------------------------- full-size layers
+
+@pytest.mark.parametrize("name", ["B", "C", "D", "E"])
+def test_full_size_layer_parity(name):
+    layer = S.generate(S.CONFIGS[name], threads=16)
+    q, k, v = device_layer(layer)
+    cfg = make_cfg(layer)
+    ocfg = oracle_cfg(cfg)
+    host, _ = gpu_select(q, k, cfg)
+    oidx = oracle_heads(layer, ocfg)
+    rep = P.Report()
+    check_index(host, oidx, cfg, rep)
+    rep.assert_ok()
+    # planted structure must be selected, Gaussian heads must route PE
+    for h in layer.planted_q_heads:
+        assert host["route"][h] == O.VS
+        st = layer.structure[h // layer.cfg.group]
+        assert host["sel_v"][h][st.verticals // 128].all()
+        assert host["sel_s"][h][st.slash_offsets // 128].all()
+    for h in layer.gaussian_q_heads:
+        assert host["route"][h] == O.PE
+    out = torch.empty_like(q)
+    crisp.prefill(q, k, v, out, cfg)
+    crisp.raise_on_device_status(cfg, where="prefill")
+    rows = sample_rows(cfg.n, cfg.n_blocks, full=False)
+    check_outputs(layer, out, oidx, ocfg, rows, skip_heads=rep.heads_with_flips())

@@ -1,0 +1,47 @@
+"""Host-side comparison rules used by the GPU parity tests (no GPU needed)."""
+import numpy as np
+
+import parity as P
+from oracle import crisp_oracle as O
+
+
+def test_mask_pack_roundtrip():
+    r = np.random.default_rng(0)
+    for nb in (1, 31, 32, 33, 100, 4096):
+        bits = r.random((3, nb)) < 0.4
+        words = P.pack_mask(bits)
+        assert words.shape == (3, (nb + 31) // 32)
+        assert (P.unpack_mask(words, nb) == bits).all()
+    w = P.pack_mask(np.array([True, False, True] + [False] * 29 + [True]))
+    assert w.tolist() == [5, 1]
+
+
+def _idx(route=O.VS, c=0.5):
+    p = np.array([0.4, 0.05, 0.2, 0.05, 0.3])
+    sel, mu = O.threshold_blocks(p, 0, 4, 1.0)
+    return O.HeadIndex(c, route, p, p.copy(), sel, sel.copy(), mu, mu, None)
+
+
+def test_route_flip_only_near_tau():
+    rep = P.Report()
+    P.compare_route(0, 0.5, O.PE, _idx(c=0.5), 0.1, rep)
+    assert rep.failures
+    rep = P.Report()
+    P.compare_route(0, 0.10001, O.PE, _idx(c=0.10001), 0.1, rep)
+    assert rep.route_flips == [0] and not rep.failures
+
+
+def test_vs_mismatch_far_from_threshold_fails_near_is_flip():
+    idx = _idx()
+    gpu = idx.sel_v.copy()
+    gpu[1] = True                     # p=0.05 vs thr=0.1: far -> failure
+    rep = P.Report()
+    P.compare_vs(0, gpu, idx.sel_s, idx, 1.0, rep)
+    assert rep.failures
+    idx.p_v[1] = idx.mu_v * (1 + 1e-4)  # now within 1e-3 of the threshold -> flip
+    idx.sel_v[1] = True
+    gpu2 = idx.sel_v.copy()
+    gpu2[1] = False
+    rep = P.Report()
+    P.compare_vs(0, gpu2, idx.sel_s, idx, 1.0, rep)
+    assert not rep.failures and rep.vs_flips[0] == 1
