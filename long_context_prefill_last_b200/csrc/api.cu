@@ -174,7 +174,10 @@ static IndexPtrs from_abi(const crisp_index* ix) {
 static crisp_status run_index(const void* q, const void* k, const Shape& s, char* ws, const WsLayout& L,
                               const IndexPtrs& ix, bool with_pe, cudaStream_t st) {
   CRISP_TRY(cudaMemsetAsync(ws + L.kv_pe, 0, (size_t)s.h_kv * 4, st));
-  CRISP_TRY(launch_proxy_simt(q, k, s, ws, L, st));
+  if (!s.fp32 && use_tensor_cores())
+    CRISP_TRY(launch_proxy_tc(q, k, s, ws, L, st));
+  else
+    CRISP_TRY(launch_proxy_simt(q, k, s, ws, L, st));
   CRISP_TRY(launch_finalize(s, ws, L, ix, st));
   CRISP_TRY(launch_vs_select(s, ws, L, ix, st));
   if (with_pe) CRISP_TRY(launch_pe(q, k, s, ws, L, ix, st));

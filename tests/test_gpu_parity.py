@@ -231,6 +231,23 @@ def test_tensor_core_and_cuda_core_attention_agree():
         assert err < 2e-2
 
 
+@pytest.mark.parametrize("base,n,hq,hkv", [("B", 4096, 8, 2), ("D", 2048, 14, 2), ("B", 640, 1, 1)])
+def test_tensor_core_and_cuda_core_proxy_agree(base, n, hq, hkv):
+    layer = S.generate(S.scaled(base, n=n, h_q=hq, h_kv=hkv))
+    q, k, _ = device_layer(layer)
+    cfg = make_cfg(layer)
+    res = []
+    for force in ("0", "1"):
+        os.environ["CRISP_FORCE_SIMT"] = force
+        try:
+            host, _ = gpu_select(q, k, cfg)
+            res.append(host)
+        finally:
+            os.environ.pop("CRISP_FORCE_SIMT", None)
+    for f in ("p_v", "p_s", "c_struct"):
+        np.testing.assert_allclose(res[0][f], res[1][f], rtol=1e-4, atol=1e-7)
+
+
 def test_repeat_calls_are_deterministic():
     layer = S.generate(S.scaled("D", n=2048, h_q=14, h_kv=2))
     q, k, v = device_layer(layer)
