@@ -6,15 +6,20 @@
 // element-exactly inside a tile. The same kernel with every causal tile kept
 // is the dense reference.
 //
-// One CTA per (query tile of 128 rows, query head); 6 warps:
-//   warp 0      TMA producer: Q once, then K and V tiles through 2-stage rings
+// One CTA per (pair of adjacent 128-row query tiles A = I, B = I-1, query
+// head); the K/V tiles of the union of their schedules stream once through
+// shared memory and serve both. 10 warps:
+//   warp 0      TMA producer: Q_A, Q_B once, then K (3-stage ring) and V (2-stage ring)
 //   warp 1      TMEM allocation; one thread issues every tcgen05.mma
-//   warps 2..5  softmax: one query row per thread (TMEM lane = row)
-// TMEM columns: S double buffer [0,128) [128,256), O [256,384).
-// Per kept tile k:  S[k%2] = Q K_k^T  ->  softmax -> P[k%2] (bf16, smem)
-//                   O += P[k%2] V_k.   S(k+1) is computed while row k's
-// softmax runs. O is rescaled lazily: only when a row's running maximum grows
-// by more than 2^8, after the previous P V has landed.
+//   warps 2..5  softmax of tile A, warps 6..9 softmax of tile B (row = TMEM lane)
+// TMEM (512 columns): S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512).
+// P (bf16) is written back over the first 64 columns of S and read by the
+// P.V MMA straight from TMEM. MMA issue order per kept tile u:
+//     S_B(u) = Q_B K_u^T,  O_A += P_A(u) V_u,  S_A(u+1) = Q_A K_{u+1}^T,  O_B += P_B(u) V_u
+// so each softmax runs while the tensor pipe does two MMAs of the other tile.
+// Because MMAs complete in issue order, S_X(u) landing means O_X already holds
+// P_X(u-1) V: the softmax may rescale O_X without another wait. Rescaling is
+// lazy: only when a row's running maximum grows by more than 2^8.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
@@ -26,41 +31,38 @@
 namespace crisp {
 namespace {
 
-constexpr int kThreads = 192;
-constexpr int kStages = 2;
+constexpr int kThreads = 320;
+constexpr int kKStages = 3;
+constexpr int kVStages = 2;
 constexpr uint32_t kTileBytes = 128 * 128 * 2;   // one bf16 128x128 tile (two 64-column halves)
 constexpr uint32_t kHalfBytes = 128 * 128;       // one half: 128 rows x 128 bytes
-constexpr uint32_t OFF_Q = 0;
-constexpr uint32_t OFF_K = OFF_Q + kTileBytes;
-constexpr uint32_t OFF_V = OFF_K + kStages * kTileBytes;
-constexpr uint32_t OFF_P = OFF_V + kStages * kTileBytes;
-constexpr uint32_t OFF_BAR = OFF_P + 2 * kTileBytes;
-// barriers (8 bytes each)
+constexpr uint32_t OFF_QA = 0;
+constexpr uint32_t OFF_QB = kTileBytes;
+constexpr uint32_t OFF_K = 2 * kTileBytes;
+constexpr uint32_t OFF_V = OFF_K + kKStages * kTileBytes;
+constexpr uint32_t OFF_BAR = OFF_V + kVStages * kTileBytes;
 enum {
   B_Q = 0,
   B_KFULL = 1,
-  B_KEMPTY = B_KFULL + kStages,
-  B_VFULL = B_KEMPTY + kStages,
-  B_VEMPTY = B_VFULL + kStages,
-  B_SFULL = B_VEMPTY + kStages,
-  B_SEMPTY = B_SFULL + 2,
-  B_PFULL = B_SEMPTY + 2,
-  B_PVDONE = B_PFULL + 2,
-  B_DRAIN = B_PVDONE + 2,
+  B_KEMPTY = B_KFULL + kKStages,
+  B_VFULL = B_KEMPTY + kKStages,
+  B_VEMPTY = B_VFULL + kVStages,
+  B_SFULL = B_VEMPTY + kVStages,   // [2]: S_X landed
+  B_PFULL = B_SFULL + 2,           // [2]: P_X written (128 arrivals)
+  B_DONE = B_PFULL + 2,            // [2]: last P_X V landed
+  B_DRAIN = B_DONE + 2,
   B_COUNT = B_DRAIN + 1
 };
 constexpr uint32_t OFF_TMEMPTR = OFF_BAR + 8 * B_COUNT;
 constexpr uint32_t OFF_ABORT = OFF_TMEMPTR + 4;
-constexpr uint32_t kSmemUsed = OFF_ABORT + 4;
-constexpr uint32_t kSmemBytes = kSmemUsed + 1024;   // slack to align the base to 1024
+constexpr uint32_t kSmemBytes = OFF_ABORT + 4 + 1024;   // + slack to align the base to 1024
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t TM_S0 = 0, TM_O = 256;
 constexpr float kRescaleLog2 = 8.f;
 
 struct TcArgs {
-  int n, nb, words, group, h_q;
+  int n, nb, words, group, h_q, n_pairs;
   float scale_log2;
   int dense;
   const int32_t* route;
@@ -72,12 +74,45 @@ struct TcArgs {
 
 __device__ __forceinline__ uint32_t bar_addr(uint32_t base, int i) { return base + OFF_BAR + 8u * i; }
 
-// Every lane waits; the warp proceeds only if all lanes saw the phase complete,
-// so warp-collective tcgen05 loads and stores never run on a diverged warp.
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag, int32_t* status,
                                           int where) {
   const bool ok = dev::mbar_wait(bar, parity, abort_flag, status, where);
   return __all_sync(0xffffffffu, ok);
+}
+
+// The two query tiles' schedules (same head, tiles IA and IB = IA - 1).
+struct Sched {
+  int IA, IB, route;
+  bool dense;
+  const uint32_t *vmask, *smask, *peA, *peB;
+  __device__ int kindA(int t) const { return dev::tile_kind(route, vmask, smask, peA, dense, IA, t); }
+  __device__ int kindB(int t) const {
+    return (IB >= 0 && t <= IB) ? dev::tile_kind(route, vmask, smask, peB, dense, IB, t) : (int)dev::kSkip;
+  }
+  // next tile >= t needed by A or B; returns false at the end
+  __device__ bool next(int& t, int& ka, int& kb) const {
+    for (; t <= IA; ++t) {
+      ka = kindA(t);
+      kb = kindB(t);
+      if (ka != dev::kSkip || kb != dev::kSkip) return true;
+    }
+    return false;
+  }
+};
+
+// Kept columns of a row: all (full tile), c <= r (lower) or c > r (upper).
+__device__ __forceinline__ void mask_row(float (&s)[128], int kind, int r) {
+  if (kind == dev::kLower) {
+#pragma unroll
+    for (int c = 0; c < 128; ++c) s[c] = c <= r ? s[c] : -INFINITY;
+  } else if (kind == dev::kUpper) {
+#pragma unroll
+    for (int c = 0; c < 128; ++c) s[c] = c > r ? s[c] : -INFINITY;
+  }
+}
+
+__device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile_base, int kk) {
+  return dev::smem_desc_sw128(tile_base + (kk >> 2) * kHalfBytes + (kk & 3) * 32, 16, 1024);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -91,31 +126,35 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   uint32_t* tmem_ptr_smem = reinterpret_cast<uint32_t*>(sgen + OFF_TMEMPTR);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int lin = blockIdx.x;
-  const int h = lin % a.h_q;
-  const int I = (a.nb - 1) - lin / a.h_q;     // heaviest query tiles first
+  const int h = blockIdx.x % a.h_q;
+  const int pair = blockIdx.x / a.h_q;                   // heaviest pairs first
+  Sched sc;
+  sc.IA = (a.nb - 1) - 2 * pair;
+  sc.IB = sc.IA - 1;
+  sc.dense = a.dense != 0;
+  sc.route = sc.dense ? 0 : a.route[h];
+  sc.vmask = a.vs_mask + (size_t)h * 2 * a.words;
+  sc.smask = sc.vmask + a.words;
+  sc.peA = a.pe_mask + ((size_t)h * a.nb + sc.IA) * a.words;
+  sc.peB = a.pe_mask + ((size_t)h * a.nb + (sc.IB >= 0 ? sc.IB : 0)) * a.words;
   const int g = h / a.group;
-  const int route = a.dense ? 0 : a.route[h];
-  const uint32_t* vmask = a.vs_mask + (size_t)h * 2 * a.words;
-  const uint32_t* smask = vmask + a.words;
-  const uint32_t* pe_row = a.pe_mask + ((size_t)h * a.nb + I) * a.words;
-  const bool dense = a.dense != 0;
+  const bool hasB = sc.IB >= 0;
 
   if (threadIdx.x == 0) {
-    // an earlier failure anywhere in the grid: this CTA does nothing
-    *abort_flag = dev::load_volatile(a.status) != 0 ? 1 : 0;
+    *abort_flag = dev::load_volatile(a.status) != 0 ? 1 : 0;   // an earlier failure: do nothing
     dev::mbar_init(bar_addr(sbase, B_Q), 1);
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kKStages; ++s) {
       dev::mbar_init(bar_addr(sbase, B_KFULL + s), 1);
       dev::mbar_init(bar_addr(sbase, B_KEMPTY + s), 1);
+    }
+    for (int s = 0; s < kVStages; ++s) {
       dev::mbar_init(bar_addr(sbase, B_VFULL + s), 1);
       dev::mbar_init(bar_addr(sbase, B_VEMPTY + s), 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      dev::mbar_init(bar_addr(sbase, B_SFULL + b), 1);
-      dev::mbar_init(bar_addr(sbase, B_SEMPTY + b), 128);
-      dev::mbar_init(bar_addr(sbase, B_PFULL + b), 128);
-      dev::mbar_init(bar_addr(sbase, B_PVDONE + b), 1);
+    for (int x = 0; x < 2; ++x) {
+      dev::mbar_init(bar_addr(sbase, B_SFULL + x), 1);
+      dev::mbar_init(bar_addr(sbase, B_PFULL + x), 128);
+      dev::mbar_init(bar_addr(sbase, B_DONE + x), 1);
     }
     dev::mbar_init(bar_addr(sbase, B_DRAIN), 1);
     dev::fence_mbar_init();
@@ -132,25 +171,27 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   const uint32_t tmem = *tmem_ptr_smem;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
+    // ---------------------------------------------------------------- TMA producer
     if (lane == 0) {
       dev::prefetch_tmap(&tm_q);
       dev::prefetch_tmap(&tm_k);
       dev::prefetch_tmap(&tm_v);
       const uint32_t bq = bar_addr(sbase, B_Q);
-      dev::mbar_arrive_expect_tx(bq, kTileBytes);
-      dev::tma_load_3d(sbase + OFF_Q, &tm_q, bq, 0, I * 128, h);
-      dev::tma_load_3d(sbase + OFF_Q + kHalfBytes, &tm_q, bq, 64, I * 128, h);
-      int k = 0, prev_t = -1;
+      dev::mbar_arrive_expect_tx(bq, hasB ? 2 * kTileBytes : kTileBytes);
+      dev::tma_load_3d(sbase + OFF_QA, &tm_q, bq, 0, sc.IA * 128, h);
+      dev::tma_load_3d(sbase + OFF_QA + kHalfBytes, &tm_q, bq, 64, sc.IA * 128, h);
+      if (hasB) {
+        dev::tma_load_3d(sbase + OFF_QB, &tm_q, bq, 0, sc.IB * 128, h);
+        dev::tma_load_3d(sbase + OFF_QB + kHalfBytes, &tm_q, bq, 64, sc.IB * 128, h);
+      }
+      int u = 0, t = 0, ka = 0, kb = 0, prev_t = -1;
       int issued_k = 0, issued_v = 0;
-      bool ok = true;
-      for (int t = 0; t <= I + 1 && ok; ++t) {
-        int kind = dev::kSkip;
-        if (t <= I) kind = dev::tile_kind(route, vmask, smask, pe_row, dense, I, t);
-        if (t <= I && kind == dev::kSkip) continue;
-        if (t <= I) {   // K of tile k
-          const int s = k % kStages;
-          if (!dev::mbar_wait(bar_addr(sbase, B_KEMPTY + s), ((k / kStages) & 1) ^ 1, abort_flag, a.status, 1)) {
+      bool ok = true, more = true;
+      while (ok && (more || prev_t >= 0)) {
+        more = more && sc.next(t, ka, kb);
+        if (more) {   // K of tile u
+          const int s = u % kKStages;
+          if (!dev::mbar_wait(bar_addr(sbase, B_KEMPTY + s), ((u / kKStages) & 1) ^ 1, abort_flag, a.status, 1)) {
             ok = false;
             break;
           }
@@ -160,9 +201,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           dev::tma_load_3d(sbase + OFF_K + s * kTileBytes + kHalfBytes, &tm_k, bk, 64, t * 128, g);
           ++issued_k;
         }
-        if (k >= 1) {   // V of tile k-1
-          const int kv = k - 1, s = kv % kStages;
-          if (!dev::mbar_wait(bar_addr(sbase, B_VEMPTY + s), ((kv / kStages) & 1) ^ 1, abort_flag, a.status, 2)) {
+        if (prev_t >= 0) {   // V of tile u-1
+          const int uv = u - 1, s = uv % kVStages;
+          if (!dev::mbar_wait(bar_addr(sbase, B_VEMPTY + s), ((uv / kVStages) & 1) ^ 1, abort_flag, a.status, 2)) {
             ok = false;
             break;
           }
@@ -172,192 +213,215 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           dev::tma_load_3d(sbase + OFF_V + s * kTileBytes + kHalfBytes, &tm_v, bv, 64, prev_t * 128, g);
           ++issued_v;
         }
-        prev_t = t;
-        ++k;
+        prev_t = more ? t : -1;
+        if (more) {
+          ++t;
+          ++u;
+        }
       }
       if (!ok) {
         // error path: let the copies already issued land before the CTA exits
         dev::mbar_drain(bq, 0);
-        for (int s = 0; s < kStages; ++s) {
-          const int last_k = issued_k - 1 - ((issued_k - 1 - s) % kStages + kStages) % kStages;
-          if (issued_k > s && last_k >= 0) dev::mbar_drain(bar_addr(sbase, B_KFULL + s), (last_k / kStages) & 1);
-          const int last_v = issued_v - 1 - ((issued_v - 1 - s) % kStages + kStages) % kStages;
-          if (issued_v > s && last_v >= 0) dev::mbar_drain(bar_addr(sbase, B_VFULL + s), (last_v / kStages) & 1);
+        for (int s = 0; s < kKStages && s < issued_k; ++s) {
+          const int last = issued_k - 1 - ((issued_k - 1 - s) % kKStages);
+          dev::mbar_drain(bar_addr(sbase, B_KFULL + s), (last / kKStages) & 1);
+        }
+        for (int s = 0; s < kVStages && s < issued_v; ++s) {
+          const int last = issued_v - 1 - ((issued_v - 1 - s) % kVStages);
+          dev::mbar_drain(bar_addr(sbase, B_VFULL + s), (last / kVStages) & 1);
         }
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+    // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       const uint32_t idesc_qk = dev::umma_idesc_bf16(128, 128, false);
       const uint32_t idesc_pv = dev::umma_idesc_bf16(128, 128, true);
-      bool ok = dev::mbar_wait(bar_addr(sbase, B_Q), 0, abort_flag, a.status, 3);
-      dev::tc_fence_after();
-      int k = 0;
-      auto issue_pv = [&](int kp) -> bool {
-        const int pb = kp & 1, s = kp % kStages;
-        if (!dev::mbar_wait(bar_addr(sbase, B_PFULL + pb), (kp >> 1) & 1, abort_flag, a.status, 4)) return false;
-        if (!dev::mbar_wait(bar_addr(sbase, B_VFULL + s), (kp / kStages) & 1, abort_flag, a.status, 5)) return false;
-        dev::tc_fence_after();
-        const uint32_t p_base = sbase + OFF_P + pb * kTileBytes;
-        const uint32_t v_base = sbase + OFF_V + s * kTileBytes;
+      const uint32_t S[2] = {tmem + 0u, tmem + 128u};
+      const uint32_t O[2] = {tmem + 256u, tmem + 384u};
+      const uint32_t QS[2] = {sbase + OFF_QA, sbase + OFF_QB};
+      int kx[2] = {0, 0};   // P.V issued per tile
+      auto qk = [&](int x, int u) {
+        const uint32_t kb = sbase + OFF_K + (u % kKStages) * kTileBytes;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t ad = dev::smem_desc_sw128(p_base + (kk >> 2) * kHalfBytes + (kk & 3) * 32, 16, 1024);
-          const uint64_t bd = dev::smem_desc_sw128(v_base + kk * 2048, kHalfBytes, 1024);
-          dev::umma_ss(tmem + TM_O, ad, bd, idesc_pv, (kp > 0 || kk > 0) ? 1u : 0u);
-        }
-        dev::umma_commit(bar_addr(sbase, B_PVDONE + pb));
-        dev::umma_commit(bar_addr(sbase, B_VEMPTY + s));
+        for (int kk = 0; kk < 8; ++kk)
+          dev::umma_ss(S[x], kmajor_desc(QS[x], kk), kmajor_desc(kb, kk), idesc_qk, kk > 0 ? 1u : 0u);
+        dev::umma_commit(bar_addr(sbase, B_SFULL + x));
+      };
+      auto pv = [&](int x, int u) -> bool {
+        if (!dev::mbar_wait(bar_addr(sbase, B_PFULL + x), kx[x] & 1, abort_flag, a.status, 4 + x)) return false;
+        dev::tc_fence_after();
+        const uint32_t vb = sbase + OFF_V + (u % kVStages) * kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          dev::umma_ts(O[x], S[x] + kk * 8, dev::smem_desc_sw128(vb + kk * 2048, kHalfBytes, 1024), idesc_pv,
+                       (kx[x] > 0 || kk > 0) ? 1u : 0u);
+        ++kx[x];
         return true;
       };
-      for (int t = 0; t <= I && ok; ++t) {
-        const int kind = dev::tile_kind(route, vmask, smask, pe_row, dense, I, t);
-        if (kind == dev::kSkip) continue;
-        const int s = k % kStages, sb = k & 1;
-        if (!dev::mbar_wait(bar_addr(sbase, B_KFULL + s), (k / kStages) & 1, abort_flag, a.status, 6)) {
-          ok = false;
-          break;
-        }
-        if (k >= 2 &&
-            !dev::mbar_wait(bar_addr(sbase, B_SEMPTY + sb), ((k - 2) >> 1) & 1, abort_flag, a.status, 7)) {
+      bool ok = dev::mbar_wait(bar_addr(sbase, B_Q), 0, abort_flag, a.status, 3);
+      int t = 0, ka = 0, kb = 0;
+      bool have = ok && sc.next(t, ka, kb);
+      if (have) {
+        ok = dev::mbar_wait(bar_addr(sbase, B_KFULL + 0), 0, abort_flag, a.status, 6);
+        dev::tc_fence_after();
+        if (ok && ka != dev::kSkip) qk(0, 0);
+      }
+      int u = 0;
+      while (ok && have) {
+        // lookahead: the tile after u
+        int t2 = t + 1, ka2 = 0, kb2 = 0;
+        const bool have2 = sc.next(t2, ka2, kb2);
+        if (kb != dev::kSkip) qk(1, u);
+        dev::umma_commit(bar_addr(sbase, B_KEMPTY + u % kKStages));
+        if (!dev::mbar_wait(bar_addr(sbase, B_VFULL + u % kVStages), (u / kVStages) & 1, abort_flag, a.status, 7)) {
           ok = false;
           break;
         }
         dev::tc_fence_after();
-        const uint32_t k_base = sbase + OFF_K + s * kTileBytes;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-          const uint64_t ad = dev::smem_desc_sw128(sbase + OFF_Q + off, 16, 1024);
-          const uint64_t bd = dev::smem_desc_sw128(k_base + off, 16, 1024);
-          dev::umma_ss(tmem + TM_S0 + sb * 128, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
-        }
-        dev::umma_commit(bar_addr(sbase, B_SFULL + sb));
-        dev::umma_commit(bar_addr(sbase, B_KEMPTY + s));
-        if (k >= 1 && !issue_pv(k - 1)) {
+        if (ka != dev::kSkip && !pv(0, u)) {
           ok = false;
           break;
         }
-        ++k;
+        if (have2) {
+          if (!dev::mbar_wait(bar_addr(sbase, B_KFULL + (u + 1) % kKStages), ((u + 1) / kKStages) & 1, abort_flag,
+                              a.status, 8)) {
+            ok = false;
+            break;
+          }
+          dev::tc_fence_after();
+          if (ka2 != dev::kSkip) qk(0, u + 1);
+        }
+        if (kb != dev::kSkip && !pv(1, u)) {
+          ok = false;
+          break;
+        }
+        dev::umma_commit(bar_addr(sbase, B_VEMPTY + u % kVStages));
+        t = t2;
+        ka = ka2;
+        kb = kb2;
+        have = have2;
+        ++u;
       }
-      if (ok && k >= 1) ok = issue_pv(k - 1);
-      // all MMAs issued must complete before TMEM is released
+      if (ok) {
+        dev::umma_commit(bar_addr(sbase, B_DONE + 0));
+        dev::umma_commit(bar_addr(sbase, B_DONE + 1));
+      }
+      // every MMA issued must complete before TMEM is released
       dev::umma_commit(bar_addr(sbase, B_DRAIN));
       dev::mbar_drain(bar_addr(sbase, B_DRAIN), 0);
     }
   } else {
-    // ------------------------------------------------------------ softmax warps
-    const int quarter = warp & 3;                 // TMEM lane quarter this warp may access
+    // ---------------------------------------------------------------- softmax warps
+    const int x = (warp - 2) >> 2;                // 0: tile A, 1: tile B
+    const int quarter = warp & 3;                 // TMEM lane quarter of this warp
     const int r = quarter * 32 + lane;            // query row inside the tile
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-    float m_ref = -INFINITY, l = 0.f;
-    int k = 0;
-    bool ok = true;
-    for (int t = 0; t <= I; ++t) {
-      const int kind = dev::tile_kind(route, vmask, smask, pe_row, dense, I, t);
-      if (kind == dev::kSkip) continue;
-      const int sb = k & 1;
-      if (!warp_wait(bar_addr(sbase, B_SFULL + sb), (k >> 1) & 1, abort_flag, a.status, 8)) {
-        ok = false;
-        break;
-      }
-      dev::tc_fence_after();
-      float x[128];
-#pragma unroll
-      for (int c0 = 0; c0 < 128; c0 += 32) {
-        uint32_t v[32];
-        dev::tmem_ld32(tmem + lane_base + TM_S0 + sb * 128 + c0, v);
-        dev::tmem_wait_ld();
-#pragma unroll
-        for (int j = 0; j < 32; ++j) x[c0 + j] = __uint_as_float(v[j]);
-      }
-      dev::tc_fence_before();
-      dev::mbar_arrive(bar_addr(sbase, B_SEMPTY + sb));
-      float tmax = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        const bool keep = kind == dev::kFull || (kind == dev::kLower ? c <= r : c > r);
-        x[c] = keep ? x[c] * a.scale_log2 : -INFINITY;
-        tmax = fmaxf(tmax, x[c]);
-      }
-      const bool need = tmax > m_ref + kRescaleLog2;
-      const float m_new = need ? tmax : m_ref;
-      const float factor = need ? dev::ex2(m_ref - m_new) : 1.f;   // 0 when m_ref = -inf
-      if (k > 0 && __any_sync(0xffffffffu, need)) {
-        // O holds P V up to tile k-1: wait for it, then scale this warp's rows
-        const int kp = k - 1;
-        if (!warp_wait(bar_addr(sbase, B_PVDONE + (kp & 1)), (kp >> 1) & 1, abort_flag, a.status, 9)) {
+    const uint32_t s_col = tmem + lane_base + (uint32_t)x * 128;
+    const uint32_t o_col = tmem + lane_base + 256u + (uint32_t)x * 128;
+    const int I = x == 0 ? sc.IA : sc.IB;
+    if (I >= 0) {
+      const float sl2 = a.scale_log2;
+      float m_ref = -INFINITY, l = 0.f;
+      int k = 0;
+      bool ok = true;
+      for (int t = 0; t <= I; ++t) {
+        const int kind = x == 0 ? sc.kindA(t) : sc.kindB(t);
+        if (kind == dev::kSkip) continue;
+        if (!warp_wait(bar_addr(sbase, B_SFULL + x), k & 1, abort_flag, a.status, 10 + x)) {
           ok = false;
           break;
         }
         dev::tc_fence_after();
+        // pass 1: row maximum over the kept columns
+        float tmax;
+        {
+          float s[128];
+          dev::tmem_ld128(s_col, s);
+          dev::tmem_wait_ld();
+          mask_row(s, kind, r);
+          float mx[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) mx[j] = s[j];
+#pragma unroll
+          for (int c = 8; c < 128; ++c) mx[c & 7] = fmaxf(mx[c & 7], s[c]);
+          tmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                       fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sl2;
+        }
+        const bool need = tmax > m_ref + kRescaleLog2;
+        const float factor = need ? dev::ex2(m_ref - tmax) : 1.f;   // 0 when m_ref = -inf
+        if (k > 0 && __any_sync(0xffffffffu, need)) {
+          // O holds P V of every earlier tile (it completed before S landed)
+#pragma unroll 1
+          for (int c0 = 0; c0 < 128; c0 += 32) {
+            uint32_t v[32];
+            dev::tmem_ld32(o_col + c0, v);
+            dev::tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * factor);
+            dev::tmem_st32(o_col + c0, v);
+          }
+        }
+        if (need) {
+          l *= factor;
+          m_ref = tmax;
+        }
+        const float neg_m = m_ref == -INFINITY ? 0.f : -m_ref;
+        // pass 2: P = 2^(s*scale - m) in 32-column chunks; chunk j of P (bf16
+        // pairs) goes to S columns [16j, 16j+16), which pass 2 has already read.
+        float sum[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) sum[j] = 0.f;
 #pragma unroll
         for (int c0 = 0; c0 < 128; c0 += 32) {
-          uint32_t v[32];
-          dev::tmem_ld32(tmem + lane_base + TM_O + c0, v);
+          float s[32];
+          dev::tmem_ld32(s_col + c0, reinterpret_cast<uint32_t (&)[32]>(s));
           dev::tmem_wait_ld();
+          if (kind != dev::kFull) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * factor);
-          dev::tmem_st32(tmem + lane_base + TM_O + c0, v);
+            for (int j = 0; j < 32; ++j) {
+              const int c = c0 + j;
+              const bool keep = kind == dev::kLower ? c <= r : c > r;
+              s[j] = keep ? s[j] : -INFINITY;
+            }
+          }
+          uint32_t pk[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const float p0 = dev::ex2(fmaf(s[2 * j], sl2, neg_m));
+            const float p1 = dev::ex2(fmaf(s[2 * j + 1], sl2, neg_m));
+            sum[(2 * j) & 7] += p0;
+            sum[(2 * j + 1) & 7] += p1;
+            pk[j] = dev::pack_bf16x2(p0, p1);
+          }
+          dev::tmem_st16(s_col + (c0 >> 1), pk);
         }
         dev::tmem_wait_st();
         dev::tc_fence_before();
+        dev::mbar_arrive(bar_addr(sbase, B_PFULL + x));
+        l += ((sum[0] + sum[1]) + (sum[2] + sum[3])) + ((sum[4] + sum[5]) + (sum[6] + sum[7]));
+        ++k;
       }
-      l *= factor;
-      m_ref = m_new;
-      const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
-      // P = 2^(x - m), row sum, packed to bf16
-      uint32_t pk[64];
-      float rs = 0.f;
+      // epilogue: O / l -> bf16 row of the output
+      if (ok && k > 0) ok = warp_wait(bar_addr(sbase, B_DONE + x), 0, abort_flag, a.status, 12 + x);
+      if (ok && k > 0) {
+        dev::tc_fence_after();
+        const float inv = 1.f / l;
+        __nv_bfloat16* orow = a.out + ((size_t)h * a.n + (size_t)I * 128 + r) * kHeadDim;
 #pragma unroll
-      for (int c = 0; c < 128; c += 2) {
-        const float p0 = dev::ex2(x[c] - m_use);
-        const float p1 = dev::ex2(x[c + 1] - m_use);
-        rs += p0 + p1;
-        pk[c >> 1] = dev::pack_bf16x2(p0, p1);
-      }
-      l += rs;
-      // the P buffer of tile k was read by P V of tile k-2
-      if (k >= 2) {
-        const int kp = k - 2;
-        if (!warp_wait(bar_addr(sbase, B_PVDONE + (kp & 1)), (kp >> 1) & 1, abort_flag, a.status, 10)) {
-          ok = false;
-          break;
+        for (int c0 = 0; c0 < 128; c0 += 32) {
+          uint32_t v[32];
+          dev::tmem_ld32(o_col + c0, v);
+          dev::tmem_wait_ld();
+          uint32_t w[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            w[j] = dev::pack_bf16x2(__uint_as_float(v[2 * j]) * inv, __uint_as_float(v[2 * j + 1]) * inv);
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            *reinterpret_cast<uint4*>(orow + c0 + 8 * j) =
+                make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
         }
-      }
-      uint8_t* prow = sgen + OFF_P + sb * kTileBytes + r * 128;
-#pragma unroll
-      for (int ch = 0; ch < 16; ++ch) {
-        const int half = ch >> 3, cc = ch & 7;
-        uint4 val = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
-        *reinterpret_cast<uint4*>(prow + half * kHalfBytes + ((cc ^ (r & 7)) << 4)) = val;
-      }
-      dev::fence_proxy_async_smem();
-      dev::mbar_arrive(bar_addr(sbase, B_PFULL + sb));
-      ++k;
-    }
-    // epilogue: O / l -> bf16 row of the output
-    if (ok && k > 0) {
-      const int kp = k - 1;
-      ok = warp_wait(bar_addr(sbase, B_PVDONE + (kp & 1)), (kp >> 1) & 1, abort_flag, a.status, 11);
-    }
-    if (ok && k > 0) {
-      dev::tc_fence_after();
-      const float inv = 1.f / l;
-      __nv_bfloat16* orow = a.out + ((size_t)h * a.n + (size_t)I * 128 + r) * kHeadDim;
-#pragma unroll
-      for (int c0 = 0; c0 < 128; c0 += 32) {
-        uint32_t v[32];
-        dev::tmem_ld32(tmem + lane_base + TM_O + c0, v);
-        dev::tmem_wait_ld();
-        uint32_t w[16];
-#pragma unroll
-        for (int j = 0; j < 16; ++j)
-          w[j] = dev::pack_bf16x2(__uint_as_float(v[2 * j]) * inv, __uint_as_float(v[2 * j + 1]) * inv);
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          *reinterpret_cast<uint4*>(orow + c0 + 8 * j) = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
       }
     }
     dev::tc_fence_before();
@@ -375,7 +439,8 @@ cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, void* ou
                            const int32_t* route, const uint32_t* vs_mask, const uint32_t* pe_mask, bool dense,
                            int32_t* status, cudaStream_t st) {
   CUtensorMap mq, mk, mv;
-  if (!make_bf16_map(&mq, q, s.n, s.h_q, 128) || !make_bf16_map(&mk, k, s.n, s.h_kv, 128) || !make_bf16_map(&mv, v, s.n, s.h_kv, 128))
+  if (!make_bf16_map(&mq, q, s.n, s.h_q, 128) || !make_bf16_map(&mk, k, s.n, s.h_kv, 128) ||
+      !make_bf16_map(&mv, v, s.n, s.h_kv, 128))
     return cudaErrorInvalidValue;
   TcArgs a;
   a.n = s.n;
@@ -383,6 +448,7 @@ cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, void* ou
   a.words = s.words;
   a.group = s.group;
   a.h_q = s.h_q;
+  a.n_pairs = (s.nb + 1) / 2;
   a.scale_log2 = s.scale_log2;
   a.dense = dense ? 1 : 0;
   a.route = route;
@@ -392,7 +458,7 @@ cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, void* ou
   a.status = status;
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
-  attn_tc_kernel<<<s.nb * s.h_q, kThreads, kSmemBytes, st>>>(mq, mk, mv, a);
+  attn_tc_kernel<<<a.n_pairs * s.h_q, kThreads, kSmemBytes, st>>>(mq, mk, mv, a);
   return cudaGetLastError();
 }
 

@@ -127,20 +127,48 @@ __device__ float block_reduce_sum(float v, float* sh) {
   return r;
 }
 
+__device__ float block_reduce_min(float v, float* sh) {
+  for (int o = 16; o > 0; o >>= 1) v = fminf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  if ((threadIdx.x & 31) == 0) sh[threadIdx.x >> 5] = v;
+  __syncthreads();
+  float r = INFINITY;
+  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) r = fminf(r, sh[w]);
+  __syncthreads();
+  return r;
+}
+
+constexpr int kWin = 64;   // level-0 buckets a row's values may span for the shared-memory path
+
 // Row softmax of the pooled logits, divided by N_b (the flattened map's total),
-// written in place; level-0 histogram (bits 31..20) with float64 mass.
+// written in place; level-0 histogram (bits 31..20) with float64 mass. A row's
+// values span few buckets, so counts and mass are first gathered in a
+// shared-memory window and flushed with one global atomic per bucket.
 __global__ void __launch_bounds__(256) pe_softmax_kernel(PeArgs a) {
   const int h = blockIdx.y, r = blockIdx.x;
   if (a.route[h] != 1) return;
   __shared__ float sh[32];
+  __shared__ unsigned long long wcount[kWin];
+  __shared__ double wmass[kWin];
   float* row = a.tri_buf + (size_t)h * a.tri + tri_off(r);
-  float m = -INFINITY;
-  for (int c = threadIdx.x; c <= r; c += blockDim.x) m = fmaxf(m, row[c]);
+  float m = -INFINITY, mn = INFINITY;
+  for (int c = threadIdx.x; c <= r; c += blockDim.x) {
+    m = fmaxf(m, row[c]);
+    mn = fminf(mn, row[c]);
+  }
   m = block_reduce_max(m, sh);
+  mn = block_reduce_min(mn, sh);
   float s = 0.f;
   for (int c = threadIdx.x; c <= r; c += blockDim.x) s += dev::ex2(row[c] - m);
   s = block_reduce_sum(s, sh);
   const float inv = 1.f / (s * (float)a.nb);
+  const uint32_t b_hi = __float_as_uint(dev::ex2(0.f) * inv) >> 20;      // bucket of the row maximum
+  const uint32_t b_lo = __float_as_uint(dev::ex2(mn - m) * inv) >> 20;   // bucket of the row minimum
+  const bool window = b_hi >= b_lo && b_hi - b_lo < (uint32_t)kWin;
+  for (int i = threadIdx.x; i < kWin; i += blockDim.x) {
+    wcount[i] = 0;
+    wmass[i] = 0.0;
+  }
+  __syncthreads();
   PeHist* hist = a.hist + h;
   uint32_t cur = 0xffffffffu;
   unsigned long long cnt = 0;
@@ -150,7 +178,14 @@ __global__ void __launch_bounds__(256) pe_softmax_kernel(PeArgs a) {
     row[c] = v;
     const uint32_t bucket = __float_as_uint(v) >> 20;
     if (bucket != cur) {
-      if (cur != 0xffffffffu) hist_flush(hist, cur, cnt, mass);
+      if (cnt) {
+        if (window && cur >= b_lo && cur - b_lo < (uint32_t)kWin) {
+          atomicAdd(&wcount[cur - b_lo], cnt);
+          atomicAdd(&wmass[cur - b_lo], mass);
+        } else {
+          hist_flush(hist, cur, cnt, mass);
+        }
+      }
       cur = bucket;
       cnt = 0;
       mass = 0.0;
@@ -158,7 +193,19 @@ __global__ void __launch_bounds__(256) pe_softmax_kernel(PeArgs a) {
     ++cnt;
     mass += (double)v;
   }
-  if (cur != 0xffffffffu) hist_flush(hist, cur, cnt, mass);
+  if (cnt) {
+    if (window && cur >= b_lo && cur - b_lo < (uint32_t)kWin) {
+      atomicAdd(&wcount[cur - b_lo], cnt);
+      atomicAdd(&wmass[cur - b_lo], mass);
+    } else {
+      hist_flush(hist, cur, cnt, mass);
+    }
+  }
+  __syncthreads();
+  if (window) {
+    for (int i = threadIdx.x; i < kWin; i += blockDim.x)
+      if (wcount[i]) hist_flush(hist, b_lo + i, wcount[i], wmass[i]);
+  }
 }
 
 // Histogram of the entries whose key matches the prefix found so far

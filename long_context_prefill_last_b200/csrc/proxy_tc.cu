@@ -27,7 +27,8 @@ constexpr uint32_t kTileBytes = 128 * 128 * 2;
 constexpr uint32_t kHalfBytes = 128 * 128;
 constexpr uint32_t OFF_Q = 0;                                // 2 M tiles
 constexpr uint32_t OFF_K = OFF_Q + 2 * kTileBytes;
-constexpr uint32_t OFF_BAR = OFF_K + kStages * kTileBytes;
+constexpr uint32_t OFF_PART = OFF_K + kStages * kTileBytes;   // [2*kChunkTiles][256] f32
+constexpr uint32_t OFF_BAR = OFF_PART + 2 * kChunkTiles * 256 * 4;
 enum {
   B_Q = 0,
   B_KFULL = 1,
@@ -189,82 +190,79 @@ proxy_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const int rr = (a.n - kProxyRows + ri) - (a.nb - 1) * kBlock;   // position inside the last block
     const bool active = j < heads_here;
     const int I = a.nb - 1;
+    const float sl2 = a.scale_log2;
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const size_t row = (size_t)(head0 + (active ? j : 0)) * kProxyRows + ri;
+    // this thread's chunk partials: part[(2u + {0 lo, 1 hi}) * 256 + sw*32 + lane]
+    float* part = reinterpret_cast<float*>(sgen + OFF_PART) + sw * 32 + lane;
     int k = 0;
     bool ok = true;
-    for (int c = c_begin; c < c_end && ok; ++c) {
-      float m_run = -INFINITY, l_run = 0.f;
-      float lo[kChunkTiles], hi[kChunkTiles];
-#pragma unroll
-      for (int u = 0; u < kChunkTiles; ++u) {
-        lo[u] = 0.f;
-        hi[u] = 0.f;
+    float m_run = -INFINITY, l_run = 0.f;
+    for (int t = t_begin; t < t_end && ok; ++t) {
+      const int u = (t - t_begin) % kChunkTiles;   // chunks start at t_begin (a multiple of 8)
+      const int sb = k & 1;
+      if (!warp_wait(bar_addr(sbase, B_SFULL + sb), (k >> 1) & 1, abort_flag, a.status, 25)) {
+        ok = false;
+        break;
       }
+      dev::tc_fence_after();
+      float x[128];
+      if (mt < n_mt) {
+        dev::tmem_ld128(tmem + lane_base + (uint32_t)(2 * mt + sb) * 128, x);
+        dev::tmem_wait_ld();
+      }
+      dev::tc_fence_before();
+      dev::mbar_arrive(bar_addr(sbase, B_SEMPTY + sb));
+      ++k;
+      if (active) {
+        if (t == I) {   // causal: keys after the query
 #pragma unroll
-      for (int u = 0; u < kChunkTiles; ++u) {
-        const int t = c * kChunkTiles + u;
-        if (t >= t_end) break;
-        const int sb = k & 1;
-        if (!warp_wait(bar_addr(sbase, B_SFULL + sb), (k >> 1) & 1, abort_flag, a.status, 25)) {
-          ok = false;
-          break;
+          for (int c = 64; c < 128; ++c) x[c] = c <= rr ? x[c] : -INFINITY;
         }
-        dev::tc_fence_after();
-        float x[128];
-        if (mt < n_mt) {
+        float mx[8];
 #pragma unroll
-          for (int c0 = 0; c0 < 128; c0 += 32) {
-            uint32_t v[32];
-            dev::tmem_ld32(tmem + lane_base + (uint32_t)(2 * mt + sb) * 128 + c0, v);
-            dev::tmem_wait_ld();
+        for (int q = 0; q < 8; ++q) mx[q] = x[q];
 #pragma unroll
-            for (int q = 0; q < 32; ++q) x[c0 + q] = __uint_as_float(v[q]);
-          }
-        }
-        dev::tc_fence_before();
-        dev::mbar_arrive(bar_addr(sbase, B_SEMPTY + sb));
-        ++k;
-        if (!active) continue;
-        float tmax = -INFINITY;
-#pragma unroll
-        for (int cc = 0; cc < 128; ++cc) {
-          if (t == I && cc > rr) x[cc] = -INFINITY;   // causal: keys after the query
-          tmax = fmaxf(tmax, x[cc]);
-        }
-        tmax *= a.scale_log2;
-        if (tmax > m_run + 8.f) {
+        for (int c = 8; c < 128; ++c) mx[c & 7] = fmaxf(mx[c & 7], x[c]);
+        const float tmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                 fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sl2;
+        if (tmax > m_run + 8.f) {   // lazy rescale of this chunk's partials
           const float f = dev::ex2(m_run - tmax);
           l_run *= f;
-#pragma unroll
-          for (int w = 0; w < kChunkTiles; ++w) {
-            lo[w] *= f;
-            hi[w] *= f;
+          for (int w = 0; w < u; ++w) {
+            part[(2 * w) * 256] *= f;
+            part[(2 * w + 1) * 256] *= f;
           }
           m_run = tmax;
         }
-        float slo = 0.f, shi = 0.f;
+        const float nm = -m_run;
+        float lo[4] = {0.f, 0.f, 0.f, 0.f}, hi[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int cc = 0; cc < 128; ++cc) {
-          const float p = dev::ex2(fmaf(x[cc], a.scale_log2, -m_run));
-          if (cc <= rr) slo += p; else shi += p;
+        for (int c = 0; c < 64; ++c) lo[c & 3] += dev::ex2(fmaf(x[c], sl2, nm));
+#pragma unroll
+        for (int c = 64; c < 128; ++c) {
+          const float p = dev::ex2(fmaf(x[c], sl2, nm));
+          const bool low = c <= rr;
+          lo[c & 3] += low ? p : 0.f;
+          hi[c & 3] += low ? 0.f : p;
         }
-        lo[u] = slo;
-        hi[u] = shi;
+        const float slo = (lo[0] + lo[1]) + (lo[2] + lo[3]);
+        const float shi = (hi[0] + hi[1]) + (hi[2] + hi[3]);
+        part[(2 * u) * 256] = slo;
+        part[(2 * u + 1) * 256] = shi;
         l_run += slo + shi;
-      }
-      if (ok && active) {
-        float* plo = a.part_lo + row * a.nb;
-        float* phi = a.part_hi + row * a.nb;
-#pragma unroll
-        for (int u = 0; u < kChunkTiles; ++u) {
-          const int t = c * kChunkTiles + u;
-          if (t < t_end) {
-            plo[t] = lo[u];
-            phi[t] = hi[u];
+        if (u == kChunkTiles - 1 || t == t_end - 1) {
+          const int c = t / kChunkTiles;
+          float* plo = a.part_lo + row * a.nb + (size_t)c * kChunkTiles;
+          float* phi = a.part_hi + row * a.nb + (size_t)c * kChunkTiles;
+          for (int w = 0; w <= u; ++w) {
+            plo[w] = part[(2 * w) * 256];
+            phi[w] = part[(2 * w + 1) * 256];
           }
+          a.chunk_ml[row * a.n_chunks + c] = make_float2(m_run, l_run);
+          m_run = -INFINITY;
+          l_run = 0.f;
         }
-        a.chunk_ml[row * a.n_chunks + c] = make_float2(m_run, l_run);
       }
     }
     dev::tc_fence_before();
