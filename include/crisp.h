@@ -29,7 +29,8 @@
  * - Every entry point validates its arguments before it launches anything;
  *   a failed validation returns an error and leaves memory untouched.
  * - No entry point synchronises with the host, allocates memory or keeps
- *   global mutable state. All scratch lives in the caller's workspace
+ *   global mutable state (one exception, crisp_route_noalloc, is described
+ *   at its declaration). All scratch lives in the caller's workspace
  *   (cfg.workspace, >= crisp_workspace_size bytes of device memory, 256-byte
  *   aligned). Calls that share a workspace must be ordered (same stream).
  * - `stream` is a cudaStream_t passed as a plain pointer (NULL = legacy
@@ -61,7 +62,8 @@ typedef enum {
   CRISP_ERR_CUDA = 7,          /* a CUDA runtime call or launch failed */
   CRISP_ERR_CAPACITY = 8,      /* device-side: an internal buffer would overflow */
   CRISP_ERR_TIMEOUT = 9,       /* device-side: a bounded wait ran out */
-  CRISP_ERR_NONFINITE = 10     /* device-side: a proxy statistic was NaN or infinite */
+  CRISP_ERR_NONFINITE = 10,    /* device-side: a proxy statistic was NaN or infinite */
+  CRISP_ERR_TOO_LARGE = 11     /* crisp_route_noalloc: the layer needs more scratch than its static array */
 } crisp_status;
 
 typedef enum { CRISP_BF16 = 0, CRISP_FP32 = 1 } crisp_dtype;
@@ -145,6 +147,31 @@ crisp_status crisp_device_status(const crisp_cfg* cfg, void* stream, int32_t* de
 
 /* Short English description of a status code (static storage). */
 const char* crisp_status_string(crisp_status status);
+
+/* crisp_route without caller memory. The paper has no counterpart; this is
+ * for callers that cannot give the library device memory at all: a plugin
+ * hook whose enqueue call hands over no workspace pointer, or a serving loop
+ * that forbids device allocation once it is running. It computes exactly what
+ * crisp_route computes (same kernels, same outputs), but its scratch is a
+ * static 32 MiB device array inside the library (CRISP_NOALLOC_SCRATCH_BYTES),
+ * which every GPU that loads the library holds until the process exits.
+ * - cfg->workspace and cfg->workspace_bytes are ignored; q, k, route and
+ *   c_struct are the caller's device buffers as for crisp_route.
+ * - Layers needing more scratch than the array holds (about
+ *   h_q * n / 128 * 640 bytes; e.g. 32 query heads up to n = 131072) are
+ *   rejected with CRISP_ERR_TOO_LARGE before anything is launched.
+ * - The first call on a device looks up the array's device address (once per
+ *   device, with that device current); make that first call before any
+ *   stream capture on the device.
+ * - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ * - All calls share the one array and leave their contents in it: calls that
+ *   can overlap on the GPU (different streams, or several host threads) race
+ *   and must be serialised by the caller. Device-side conditions (a bounded
+ *   wait that ran out) are recorded in the array, not in a caller workspace,
+ *   so crisp_device_status does not report them. */
+#define CRISP_NOALLOC_SCRATCH_BYTES (32u << 20)
+crisp_status crisp_route_noalloc(const void* q, const void* k, const crisp_cfg* cfg,
+                                 int32_t* route, float* c_struct, void* stream);
 
 /* Library version as major*10000 + minor*100 + patch. */
 int32_t crisp_version(void);

@@ -19,7 +19,7 @@ from typing import Optional
 
 __all__ = [
     "Config", "IndexBuffers", "CrispError", "lib", "library_path", "workspace_size", "index_dims",
-    "route", "select", "attend", "prefill", "dense_attention", "device_status", "status_string",
+    "route", "route_noalloc", "select", "attend", "prefill", "dense_attention", "device_status", "status_string",
     "BF16", "FP32", "ROUTE_AUTO", "ROUTE_VS", "ROUTE_PE", "SYMBOLS",
 ]
 
@@ -28,12 +28,12 @@ ROUTE_AUTO, ROUTE_VS, ROUTE_PE = -1, 0, 1
 STATUS_NAMES = {
     0: "CRISP_OK", 1: "CRISP_ERR_INVALID_ARG", 2: "CRISP_ERR_SHAPE", 3: "CRISP_ERR_DTYPE",
     4: "CRISP_ERR_ALIGN", 5: "CRISP_ERR_WORKSPACE", 6: "CRISP_ERR_UNSUPPORTED", 7: "CRISP_ERR_CUDA",
-    8: "CRISP_ERR_CAPACITY", 9: "CRISP_ERR_TIMEOUT", 10: "CRISP_ERR_NONFINITE",
+    8: "CRISP_ERR_CAPACITY", 9: "CRISP_ERR_TIMEOUT", 10: "CRISP_ERR_NONFINITE", 11: "CRISP_ERR_TOO_LARGE",
 }
 # every function include/crisp.h declares
 SYMBOLS = ["crisp_cfg_init", "crisp_workspace_size", "crisp_index_dims", "crisp_route", "crisp_select",
            "crisp_attend", "crisp_prefill", "crisp_dense_attention", "crisp_device_status",
-           "crisp_status_string", "crisp_version"]
+           "crisp_status_string", "crisp_version", "crisp_route_noalloc"]
 
 
 def library_path() -> str:
@@ -82,6 +82,7 @@ def lib() -> ctypes.CDLL:
         L.crisp_workspace_size.argtypes = [cfgp, ctypes.POINTER(ctypes.c_size_t)]
         L.crisp_index_dims.argtypes = [cfgp, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32)]
         L.crisp_route.argtypes = [vp, vp, cfgp, vp, vp, vp]
+        L.crisp_route_noalloc.argtypes = [vp, vp, cfgp, vp, vp, vp]
         L.crisp_select.argtypes = [vp, vp, cfgp, ctypes.POINTER(_Index), vp]
         L.crisp_attend.argtypes = [vp, vp, vp, vp, cfgp, ctypes.POINTER(_Index), vp]
         L.crisp_prefill.argtypes = [vp, vp, vp, vp, cfgp, vp]
@@ -206,6 +207,14 @@ def _stream(stream) -> Optional[int]:
 def route(q, k, cfg: Config, route_out, c_struct_out, stream=None) -> None:
     _check(lib().crisp_route(_ptr(q), _ptr(k), ctypes.byref(cfg._c()), _ptr(route_out), _ptr(c_struct_out),
                              _stream(stream)), "crisp_route")
+
+
+def route_noalloc(q, k, cfg: Config, route_out, c_struct_out, stream=None) -> None:
+    """crisp_route with the library's static scratch array instead of a workspace
+    (cfg.workspace is ignored). For callers that cannot give the library device
+    memory; concurrent calls race on the shared array."""
+    _check(lib().crisp_route_noalloc(_ptr(q), _ptr(k), ctypes.byref(cfg._c()), _ptr(route_out),
+                                     _ptr(c_struct_out), _stream(stream)), "crisp_route_noalloc")
 
 
 def select(q, k, cfg: Config, index: IndexBuffers, stream=None) -> None:

@@ -111,6 +111,8 @@ static crisp_status make_shape(const crisp_cfg* c, Shape* s) {
   return CRISP_OK;
 }
 
+crisp_status shape_from_cfg(const crisp_cfg* c, Shape* s) { return make_shape(c, s); }
+
 static crisp_status check_tensor(const void* p) {
   if (p == nullptr) return CRISP_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(p) % 16 != 0) return CRISP_ERR_ALIGN;
@@ -356,6 +358,7 @@ const char* crisp_status_string(crisp_status status) {
     case CRISP_ERR_CAPACITY: return "device buffer capacity exceeded";
     case CRISP_ERR_TIMEOUT: return "device wait timed out";
     case CRISP_ERR_NONFINITE: return "non-finite proxy statistic";
+    case CRISP_ERR_TOO_LARGE: return "layer too large for the static scratch array";
   }
   return "unknown status";
 }

@@ -50,6 +50,9 @@ struct Shape {
 
 WsLayout ws_layout(const Shape& s);
 
+// Validate a cfg and derive its Shape (the checks every entry point runs).
+crisp_status shape_from_cfg(const crisp_cfg* c, Shape* s);
+
 // Device pointers for one index set.
 struct IndexPtrs {
   int32_t* route;

@@ -134,6 +134,17 @@ def test_bad_pointers_and_workspace_fail_before_any_launch():
     assert L.crisp_select(0x10000, 0x20000, ctypes.byref(cfg._c()), None, None) == 1
 
 
+def test_route_noalloc_rejects_layers_beyond_its_static_scratch_before_any_launch():
+    L = crisp.lib()
+    big = crisp.Config(n=524288, h_q=32, h_kv=8)._c()
+    assert L.crisp_route_noalloc(0x10000, 0x20000, ctypes.byref(big), 0x30000, 0x40000, None) == 11
+    assert crisp.STATUS_NAMES[11] == "CRISP_ERR_TOO_LARGE"
+    assert "too large" in crisp.status_string(11)
+    small = crisp.Config(n=4096, h_q=4, h_kv=2)._c()
+    assert L.crisp_route_noalloc(0, 0x20000, ctypes.byref(small), 0x30000, 0x40000, None) == 1
+    assert L.crisp_route_noalloc(0x10008, 0x20000, ctypes.byref(small), 0x30000, 0x40000, None) == 4
+
+
 def test_status_strings():
     assert crisp.status_string(0) == "ok"
     assert "timed out" in crisp.status_string(9)
