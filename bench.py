@@ -283,6 +283,20 @@ def run_crisp(args, rank, world, local_rank):
     att_ms = [m.elapsed_time(b) for a, m, b in evs]
     crisp.raise_on_device_status(cfg, stream, "timed steps")
 
+    # --- timed: the route pass alone (proxy map + finalisation + route/VS masses)
+    r_out = torch.empty(c.h_q, dtype=torch.int32, device=dev)
+    c_out = torch.empty(c.h_q, dtype=torch.float32, device=dev)
+    crisp.route(q, k, cfg, r_out, c_out, stream)
+    torch.cuda.synchronize(dev)
+    rev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for a, b in rev:
+        a.record(stream)
+        crisp.route(q, k, cfg, r_out, c_out, stream)
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    route_ms = [a.elapsed_time(b) for a, b in rev]
+    crisp.raise_on_device_status(cfg, stream, "route")
+
     # --- timed: dense reference
     for _ in range(max(1, args.warmup // 2)):
         crisp.dense_attention(q, k, v, out, cfg, stream)
@@ -320,10 +334,11 @@ def run_crisp(args, rank, world, local_rank):
 
     # max over ranks
     vals = torch.tensor([statistics.mean(step_ms), statistics.mean(att_ms), statistics.mean(sel_ms),
-                         statistics.mean(dense_ms), statistics.mean(e2e_ms)], dtype=torch.float64, device=dev)
+                         statistics.mean(dense_ms), statistics.mean(e2e_ms), statistics.mean(route_ms)],
+                        dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-    step_m, att_m, sel_m, dense_m, e2e_m = vals.tolist()
+    step_m, att_m, sel_m, dense_m, e2e_m, route_m = vals.tolist()
     if rank != 0:
         return None
 
@@ -336,6 +351,20 @@ def run_crisp(args, rank, world, local_rank):
     d2h = int(out_h.numel() * out_h.element_size())
     src_hash = kernel_source_hash(["attn_tc.cu", "ptx.cuh"])
     traffic = load_traffic("attn_tc_kernel", src_hash)
+    # algorithmic HBM bytes of the route pass: K read once, proxy rows of Q,
+    # per-(row, tile) partials written and read back, chunk statistics
+    nb = cfg.n_blocks
+    rows = c.h_q * 64
+    route_bytes = (c.h_kv * c.n * c.d * 2 + rows * c.d * 2 + 2 * rows * nb * 8
+                   + rows * ((nb + 7) // 8) * 24)
+    # selection (PE heads): their Q and their groups' K pooled once, the pooled
+    # map written once and swept by the softmax (read+write), two histogram
+    # passes and the mask pass (reads), plus the PE masks written
+    n_pe = int((route == 1).sum())
+    g_pe = len({h // c.group for h in range(c.h_q) if route[h] == 1})
+    tri = nb * (nb + 1) // 2
+    pe_bytes = (n_pe + g_pe) * c.n * c.d * 2 + n_pe * tri * 4 * 6 + n_pe * nb * cfg.words * 4
+    hbm_peak = peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"])
     res = {
         "metric": METRIC,
         "value": round(step_m / world, 4),
@@ -364,6 +393,16 @@ def run_crisp(args, rank, world, local_rank):
                      "peak_source": f"{peak_src} bf16 dense, sustained (kernel runs inside a seconds-long step)",
                      "work": "4*d*128*128 flop per computed 128x128 tile x computed tiles per launch"},
         "dense_tflops": round(dense_flops / (dense_m * 1e-3) / 1e12, 2),
+        "route_roofline": {"stage": "crisp_route (proxy_tc_kernel + finalize + VS masses)", "bound": "hbm",
+                           "ms": round(route_m, 4), "algorithmic_bytes": route_bytes,
+                           "achieved": round(route_bytes / (route_m * 1e-3) / 1e9, 1), "peak": hbm_peak,
+                           "unit": "GB/s", "frac": round(route_bytes / (route_m * 1e-3) / 1e9 / hbm_peak, 4)},
+        "selection_roofline": {"stage": "PE pooling, pooled map, gamma cut, masks (select minus route)",
+                               "bound": "hbm", "ms": round(max(sel_m - route_m, 1e-6), 4),
+                               "algorithmic_bytes": pe_bytes,
+                               "achieved": round(pe_bytes / (max(sel_m - route_m, 1e-6) * 1e-3) / 1e9, 1),
+                               "peak": hbm_peak, "unit": "GB/s",
+                               "frac": round(pe_bytes / (max(sel_m - route_m, 1e-6) * 1e-3) / 1e9 / hbm_peak, 4)},
         "e2e": {"value": round(e2e_m / world, 4), "unit": "ms/layer", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "api": "crisp_prefill with pinned host buffers"},
         "gpu_launches": KERNELS_PER_STEP * args.steps,

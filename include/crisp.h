@@ -173,6 +173,12 @@ const char* crisp_status_string(crisp_status status);
 crisp_status crisp_route_noalloc(const void* q, const void* k, const crisp_cfg* cfg,
                                  int32_t* route, float* c_struct, void* stream);
 
+/* Diagnostics: evaluate, on the device, the exp2 approximations the kernels
+ * use on the FMA pipe (degree-3 and degree-5 minimax polynomials after an
+ * integer/fraction split) next to CUDA's exp2f, for n float32 inputs x
+ * (device pointers; poly3, poly5 and ref receive n values each). */
+crisp_status crisp_exp2_selftest(const float* x, float* poly3, float* poly5, float* ref, int32_t n, void* stream);
+
 /* Library version as major*10000 + minor*100 + patch. */
 int32_t crisp_version(void);
 

@@ -33,7 +33,7 @@ STATUS_NAMES = {
 # every function include/crisp.h declares
 SYMBOLS = ["crisp_cfg_init", "crisp_workspace_size", "crisp_index_dims", "crisp_route", "crisp_select",
            "crisp_attend", "crisp_prefill", "crisp_dense_attention", "crisp_device_status",
-           "crisp_status_string", "crisp_version", "crisp_route_noalloc"]
+           "crisp_status_string", "crisp_version", "crisp_route_noalloc", "crisp_exp2_selftest"]
 
 
 def library_path() -> str:
@@ -83,6 +83,7 @@ def lib() -> ctypes.CDLL:
         L.crisp_index_dims.argtypes = [cfgp, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32)]
         L.crisp_route.argtypes = [vp, vp, cfgp, vp, vp, vp]
         L.crisp_route_noalloc.argtypes = [vp, vp, cfgp, vp, vp, vp]
+        L.crisp_exp2_selftest.argtypes = [vp, vp, vp, vp, ctypes.c_int32, vp]
         L.crisp_select.argtypes = [vp, vp, cfgp, ctypes.POINTER(_Index), vp]
         L.crisp_attend.argtypes = [vp, vp, vp, vp, cfgp, ctypes.POINTER(_Index), vp]
         L.crisp_prefill.argtypes = [vp, vp, vp, vp, cfgp, vp]
@@ -235,6 +236,15 @@ def prefill(q, k, v, out, cfg: Config, stream=None) -> None:
 def dense_attention(q, k, v, out, cfg: Config, stream=None) -> None:
     _check(lib().crisp_dense_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(out), ctypes.byref(cfg._c()),
                                        _stream(stream)), "crisp_dense_attention")
+
+
+def exp2_selftest(x, stream=None):
+    """(poly3, poly5, exp2f) of a float32 CUDA tensor, evaluated on the device."""
+    import torch
+    outs = [torch.empty_like(x) for _ in range(3)]
+    _check(lib().crisp_exp2_selftest(_ptr(x), _ptr(outs[0]), _ptr(outs[1]), _ptr(outs[2]), x.numel(),
+                                     _stream(stream)), "crisp_exp2_selftest")
+    return tuple(outs)
 
 
 def device_status(cfg: Config, stream=None) -> int:

@@ -18,7 +18,7 @@ INCLUDE = os.path.join(ROOT, "include")
 OUT = os.path.join(PKG, "libcrisp.so")
 BUILD_DIR = os.path.join(ROOT, "_build")
 
-SOURCES = ["api.cu", "noalloc.cu", "proxy.cu", "proxy_tc.cu", "select.cu", "pe.cu", "attn_simt.cu", "attn_tc.cu"]
+SOURCES = ["api.cu", "noalloc.cu", "proxy.cu", "proxy_tc.cu", "select.cu", "pe.cu", "attn_simt.cu", "attn_tc.cu", "selftest.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
          "-I" + INCLUDE, "-I" + CSRC]

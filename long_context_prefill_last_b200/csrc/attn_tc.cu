@@ -8,10 +8,17 @@
 //
 // One CTA per (pair of adjacent 128-row query tiles A = I, B = I-1, query
 // head); the K/V tiles of the union of their schedules stream once through
-// shared memory and serve both. 10 warps:
-//   warp 0      TMA producer: Q_A, Q_B once, then K (3-stage ring) and V (2-stage ring)
-//   warp 1      TMEM allocation; one thread issues every tcgen05.mma
-//   warps 2..5  softmax of tile A, warps 6..9 softmax of tile B (row = TMEM lane)
+// shared memory and serve both. 12 warps in three warpgroups:
+//   warp 0       TMA producer: Q_A, Q_B once, then K (3-stage ring) and V (2-stage ring)
+//   warp 1       TMEM allocation; one thread issues every tcgen05.mma
+//   warps 2, 3   idle (they complete the first warpgroup)
+//   warps 4..7   softmax of tile A, warps 8..11 softmax of tile B (row = TMEM lane)
+// The first warpgroup gives registers to the softmax warpgroups
+// (setmaxnreg: 64 / 216 / 216 per thread; 128*64 + 256*216 <= 384*168, the
+// launch allocation), so a softmax thread holds its whole 128-column S row and
+// reads TMEM once per tile. The softmax is issue-bound as much as MUFU-bound,
+// so it uses packed f32x2 arithmetic and a three-input max, and computes one
+// exponential pair in eight on the FMA pipe (dev::exp2_poly3_x2).
 // TMEM (512 columns): S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512).
 // P (bf16) is written back over the first 64 columns of S and read by the
 // P.V MMA straight from TMEM. MMA issue order per kept tile u:
@@ -31,7 +38,10 @@
 namespace crisp {
 namespace {
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;
+constexpr int kRegsControl = 64;    // producer / MMA warpgroup after the split
+constexpr int kRegsSoftmax = 216;   // each softmax warpgroup after the split
+static_assert(128 * kRegsControl + 256 * kRegsSoftmax <= kThreads * 168, "register split exceeds the launch");
 constexpr int kKStages = 3;
 constexpr int kVStages = 2;
 constexpr uint32_t kTileBytes = 128 * 128 * 2;   // one bf16 128x128 tile (two 64-column halves)
@@ -170,6 +180,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   dev::tc_fence_after();
   const uint32_t tmem = *tmem_ptr_smem;
 
+  if (warp < 4) dev::regs_release<kRegsControl>();
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
     if (lane == 0) {
@@ -311,9 +322,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       dev::umma_commit(bar_addr(sbase, B_DRAIN));
       dev::mbar_drain(bar_addr(sbase, B_DRAIN), 0);
     }
-  } else {
+  } else if (warp >= 4) {
     // ---------------------------------------------------------------- softmax warps
-    const int x = (warp - 2) >> 2;                // 0: tile A, 1: tile B
+    dev::regs_acquire<kRegsSoftmax>();
+    const int x = (warp - 4) >> 2;                // 0: tile A, 1: tile B
     const int quarter = warp & 3;                 // TMEM lane quarter of this warp
     const int r = quarter * 32 + lane;            // query row inside the tile
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
@@ -333,21 +345,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           break;
         }
         dev::tc_fence_after();
-        // pass 1: row maximum over the kept columns
-        float tmax;
-        {
-          float s[128];
-          dev::tmem_ld128(s_col, s);
-          dev::tmem_wait_ld();
-          mask_row(s, kind, r);
-          float mx[8];
+        float s[128];
+        dev::tmem_ld128(s_col, s);
+        dev::tmem_wait_ld();
+        mask_row(s, kind, r);
+        float mx[4] = {s[0], s[1], s[2], s[3]};
 #pragma unroll
-          for (int j = 0; j < 8; ++j) mx[j] = s[j];
-#pragma unroll
-          for (int c = 8; c < 128; ++c) mx[c & 7] = fmaxf(mx[c & 7], s[c]);
-          tmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                       fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sl2;
+        for (int c = 4; c < 128; c += 8) {
+          mx[0] = dev::max3(mx[0], s[c], s[c + 1]);
+          mx[1] = dev::max3(mx[1], s[c + 2], s[c + 3]);
+          mx[2] = dev::max3(mx[2], s[c + 4], s[c + 5]);
+          mx[3] = dev::max3(mx[3], s[c + 6], s[c + 7]);
         }
+        const float tmax = fmaxf(dev::max3(mx[0], mx[1], mx[2]), mx[3]) * sl2;
         const bool need = tmax > m_ref + kRescaleLog2;
         const float factor = need ? dev::ex2(m_ref - tmax) : 1.f;   // 0 when m_ref = -inf
         if (k > 0 && __any_sync(0xffffffffu, need)) {
@@ -367,35 +377,40 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           m_ref = tmax;
         }
         const float neg_m = m_ref == -INFINITY ? 0.f : -m_ref;
-        // pass 2: P = 2^(s*scale - m) in 32-column chunks; chunk j of P (bf16
-        // pairs) goes to S columns [16j, 16j+16), which pass 2 has already read.
-        float sum[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) sum[j] = 0.f;
+        // P = 2^(s*scale - m); chunk c0 of P (bf16 pairs) goes to S columns
+        // [c0/2, c0/2 + 16), already consumed. Arguments and row sums use
+        // packed f32x2 arithmetic; one pair in eight is exponentiated on the
+        // FMA pipe, the rest on MUFU. Masked entries (-inf) give exactly 0.
+        const uint64_t scale2 = dev::f2_pack(sl2, sl2), negm2 = dev::f2_pack(neg_m, neg_m);
+        uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
         for (int c0 = 0; c0 < 128; c0 += 32) {
-          float s[32];
-          dev::tmem_ld32(s_col + c0, reinterpret_cast<uint32_t (&)[32]>(s));
-          dev::tmem_wait_ld();
-          if (kind != dev::kFull) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const int c = c0 + j;
-              const bool keep = kind == dev::kLower ? c <= r : c > r;
-              s[j] = keep ? s[j] : -INFINITY;
-            }
-          }
           uint32_t pk[16];
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
-            const float p0 = dev::ex2(fmaf(s[2 * j], sl2, neg_m));
-            const float p1 = dev::ex2(fmaf(s[2 * j + 1], sl2, neg_m));
-            sum[(2 * j) & 7] += p0;
-            sum[(2 * j + 1) & 7] += p1;
+            const int c = c0 + 2 * j;
+            const uint64_t x2 = dev::f2_fma(dev::f2_pack(s[c], s[c + 1]), scale2, negm2);
+            float p0, p1;
+            if ((j & 7) == 7) {
+              float x0, x1;
+              dev::f2_unpack(x2, x0, x1);
+              dev::exp2_poly3_x2(dev::f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f)), p0, p1);
+              p0 = s[c] == -INFINITY ? 0.f : p0;
+              p1 = s[c + 1] == -INFINITY ? 0.f : p1;
+            } else {
+              float x0, x1;
+              dev::f2_unpack(x2, x0, x1);
+              p0 = dev::ex2(x0);
+              p1 = dev::ex2(x1);
+            }
+            acc[j & 3] = dev::f2_add(acc[j & 3], dev::f2_pack(p0, p1));
             pk[j] = dev::pack_bf16x2(p0, p1);
           }
           dev::tmem_st16(s_col + (c0 >> 1), pk);
         }
+        float sum[8];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) dev::f2_unpack(acc[j], sum[2 * j], sum[2 * j + 1]);
         dev::tmem_wait_st();
         dev::tc_fence_before();
         dev::mbar_arrive(bar_addr(sbase, B_PFULL + x));

@@ -63,40 +63,60 @@ __global__ void __launch_bounds__(128) pool_kernel(const T* __restrict__ x, floa
   out[((size_t)head * nb + b) * kHeadDim + tid] = s * (1.f / kBlock);
 }
 
-// Pooled logits (log2 domain) of 16 query blocks against all key blocks c <= r.
+// Pooled logits (log2 domain) of 64 query blocks against all key blocks c <= r.
+// Tiles of 64 x 64 outputs; thread (ty, tx) holds a 4 x 4 register tile.
+// Both operand tiles sit transposed in shared memory ([d][block], row stride
+// 68 floats) so one float4 of each feeds 16 FMAs.
+constexpr int kLT = 64;       // blocks per tile side
+constexpr int kLStride = 68;  // floats per transposed row
 __global__ void __launch_bounds__(256) pe_logits_kernel(PeArgs a) {
   const int h = blockIdx.y;
   if (a.route[h] != 1) return;
   const int g = h / a.group;
-  const int r0 = blockIdx.x * 16;
-  __shared__ float qs[16][kHeadDim + 1];
-  __shared__ float ksm[64][kHeadDim + 1];
+  const int r0 = blockIdx.x * kLT;
+  extern __shared__ __align__(16) float lsm[];
+  float* qT = lsm;                        // [128][kLStride]
+  float* kT = lsm + kHeadDim * kLStride;  // [128][kLStride]
   const int tid = threadIdx.x;
-  for (int e = tid; e < 16 * kHeadDim; e += 256) {
+  for (int e = tid; e < kLT * kHeadDim; e += 256) {
     const int rr = e >> 7, dd = e & 127;
-    qs[rr][dd] = (r0 + rr < a.nb) ? a.qbar[((size_t)h * a.nb + r0 + rr) * kHeadDim + dd] * a.scale_log2 : 0.f;
+    qT[dd * kLStride + rr] =
+        (r0 + rr < a.nb) ? a.qbar[((size_t)h * a.nb + r0 + rr) * kHeadDim + dd] * a.scale_log2 : 0.f;
   }
-  const int ri = tid >> 4, cj = tid & 15;
-  const int r = r0 + ri;
-  const int rmax = min(r0 + 15, a.nb - 1);
-  for (int c0 = 0; c0 <= rmax; c0 += 64) {
+  const int ty = tid >> 4, tx = tid & 15;
+  const int rmax = min(r0 + kLT - 1, a.nb - 1);
+  for (int c0 = 0; c0 <= rmax; c0 += kLT) {
     __syncthreads();
-    for (int e = tid; e < 64 * kHeadDim; e += 256) {
+    for (int e = tid; e < kLT * kHeadDim; e += 256) {
       const int cc = e >> 7, dd = e & 127;
-      ksm[cc][dd] = (c0 + cc < a.nb) ? a.kbar[((size_t)g * a.nb + c0 + cc) * kHeadDim + dd] : 0.f;
+      kT[dd * kLStride + cc] = (c0 + cc < a.nb) ? a.kbar[((size_t)g * a.nb + c0 + cc) * kHeadDim + dd] : 0.f;
     }
     __syncthreads();
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    float acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+#pragma unroll 4
     for (int dd = 0; dd < kHeadDim; ++dd) {
-      const float qv = qs[ri][dd];
+      const float4 qv = *reinterpret_cast<const float4*>(qT + dd * kLStride + ty * 4);
+      const float4 kv = *reinterpret_cast<const float4*>(kT + dd * kLStride + tx * 4);
+      const float qa[4] = {qv.x, qv.y, qv.z, qv.w};
+      const float ka[4] = {kv.x, kv.y, kv.z, kv.w};
 #pragma unroll
-      for (int u = 0; u < 4; ++u) acc[u] = fmaf(qv, ksm[cj + 16 * u][dd], acc[u]);
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(qa[i], ka[j], acc[i][j]);
     }
-    if (r < a.nb) {
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int c = c0 + cj + 16 * u;
-        if (c <= r) a.tri_buf[(size_t)h * a.tri + tri_off(r) + c] = acc[u];
+    for (int i = 0; i < 4; ++i) {
+      const int r = r0 + ty * 4 + i;
+      if (r >= a.nb) continue;
+      float* row = a.tri_buf + (size_t)h * a.tri + tri_off(r);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int c = c0 + tx * 4 + j;
+        if (c <= r) row[c] = acc[i][j];
       }
     }
   }
@@ -471,7 +491,10 @@ cudaError_t launch_pe(const void* q, const void* k, const Shape& s, char* ws, co
     pool_kernel<__nv_bfloat16><<<dim3(s.nb, s.h_kv), 128, 0, st>>>(static_cast<const __nv_bfloat16*>(k), a.kbar,
                                                                    s.n, s.nb, a.kv_pe, 1);
   }
-  pe_logits_kernel<<<dim3((s.nb + 15) / 16, s.h_q), 256, 0, st>>>(a);
+  const size_t lsmem = 2 * kHeadDim * kLStride * sizeof(float);
+  e = cudaFuncSetAttribute(pe_logits_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lsmem);
+  if (e != cudaSuccess) return e;
+  pe_logits_kernel<<<dim3((s.nb + kLT - 1) / kLT, s.h_q), 256, lsmem, st>>>(a);
   pe_softmax_kernel<<<dim3(s.nb, s.h_q), 256, 0, st>>>(a);
   pe_find_kernel<<<s.h_q, 1024, 0, st>>>(a, 0);
   const int hist_ctas = (int)std::min<long long>(1184, (s.tri + 255) / 256);

@@ -219,13 +219,15 @@ proxy_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
           for (int c = 64; c < 128; ++c) x[c] = c <= rr ? x[c] : -INFINITY;
         }
-        float mx[8];
+        float mx[4] = {x[0], x[1], x[2], x[3]};
 #pragma unroll
-        for (int q = 0; q < 8; ++q) mx[q] = x[q];
-#pragma unroll
-        for (int c = 8; c < 128; ++c) mx[c & 7] = fmaxf(mx[c & 7], x[c]);
-        const float tmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                 fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sl2;
+        for (int c = 4; c < 128; c += 8) {
+          mx[0] = dev::max3(mx[0], x[c], x[c + 1]);
+          mx[1] = dev::max3(mx[1], x[c + 2], x[c + 3]);
+          mx[2] = dev::max3(mx[2], x[c + 4], x[c + 5]);
+          mx[3] = dev::max3(mx[3], x[c + 6], x[c + 7]);
+        }
+        const float tmax = fmaxf(dev::max3(mx[0], mx[1], mx[2]), mx[3]) * sl2;
         if (tmax > m_run + 8.f) {   // lazy rescale of this chunk's partials
           const float f = dev::ex2(m_run - tmax);
           l_run *= f;
@@ -235,19 +237,39 @@ proxy_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           }
           m_run = tmax;
         }
-        const float nm = -m_run;
-        float lo[4] = {0.f, 0.f, 0.f, 0.f}, hi[4] = {0.f, 0.f, 0.f, 0.f};
+        // exponentials with packed f32x2 arguments and sums; three pairs in
+        // eight on the FMA pipe. total = all columns, hi = columns c > rr
+        // (only in the upper half since rr >= 64); lo = total - hi holds at
+        // least the 64 lower columns, so the subtraction is well conditioned.
+        const uint64_t scale2 = dev::f2_pack(sl2, sl2), negm2 = dev::f2_pack(-m_run, -m_run);
+        uint64_t tot[4] = {0ull, 0ull, 0ull, 0ull}, hi2[2] = {0ull, 0ull};
 #pragma unroll
-        for (int c = 0; c < 64; ++c) lo[c & 3] += dev::ex2(fmaf(x[c], sl2, nm));
-#pragma unroll
-        for (int c = 64; c < 128; ++c) {
-          const float p = dev::ex2(fmaf(x[c], sl2, nm));
-          const bool low = c <= rr;
-          lo[c & 3] += low ? p : 0.f;
-          hi[c & 3] += low ? 0.f : p;
+        for (int j = 0; j < 64; ++j) {
+          const int c = 2 * j;
+          const uint64_t e2 = dev::f2_fma(dev::f2_pack(x[c], x[c + 1]), scale2, negm2);
+          float p0, p1, e0, e1;
+          dev::f2_unpack(e2, e0, e1);
+          if ((j & 7) >= 5) {
+            dev::exp2_poly3_x2(dev::f2_pack(fmaxf(e0, -125.f), fmaxf(e1, -125.f)), p0, p1);
+            if (c >= 64) {
+              p0 = x[c] == -INFINITY ? 0.f : p0;
+              p1 = x[c + 1] == -INFINITY ? 0.f : p1;
+            }
+          } else {
+            p0 = dev::ex2(e0);
+            p1 = dev::ex2(e1);
+          }
+          tot[j & 3] = dev::f2_add(tot[j & 3], dev::f2_pack(p0, p1));
+          if (c >= 64) hi2[j & 1] = dev::f2_add(hi2[j & 1], dev::f2_pack(c > rr ? p0 : 0.f, c + 1 > rr ? p1 : 0.f));
         }
-        const float slo = (lo[0] + lo[1]) + (lo[2] + lo[3]);
-        const float shi = (hi[0] + hi[1]) + (hi[2] + hi[3]);
+        float t8[8], h4[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) dev::f2_unpack(tot[q], t8[2 * q], t8[2 * q + 1]);
+        dev::f2_unpack(hi2[0], h4[0], h4[1]);
+        dev::f2_unpack(hi2[1], h4[2], h4[3]);
+        const float stot = ((t8[0] + t8[1]) + (t8[2] + t8[3])) + ((t8[4] + t8[5]) + (t8[6] + t8[7]));
+        const float shi = (h4[0] + h4[1]) + (h4[2] + h4[3]);
+        const float slo = stot - shi;
         part[(2 * u) * 256] = slo;
         part[(2 * u + 1) * 256] = shi;
         l_run += slo + shi;

@@ -240,6 +240,90 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// 2^x on the FMA and integer pipes (no MUFU). x = n + f with n = round(x):
+// adding 1.5 * 2^23 leaves round(x) in the low mantissa bits (Cody-Waite
+// style reduction), f = x - n lies in [-1/2, 1/2]; 2^f is a minimax
+// polynomial fitted by csrc/fit_exp2.py (Remez, relative error); 2^n is added
+// to the exponent field. x is clamped to >= -125 so the result stays normal.
+// Degree 3: relative error 7.5e-5 (ample for bf16 probabilities).
+__device__ __forceinline__ float exp2_poly3(float x) {
+  x = fmaxf(x, -125.f);
+  const float shifter = 12582912.f;
+  const float y = x + shifter;
+  const float f = x - (y - shifter);
+  float p = fmaf(0.0551716685f, f, 0.242611125f);
+  p = fmaf(p, f, 0.693260968f);
+  p = fmaf(p, f, 0.999928057f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(y) << 23));
+}
+
+// Degree 5: relative error 2.3e-7 in float32 (for sums that feed thresholds).
+__device__ __forceinline__ float exp2_poly5(float x) {
+  x = fmaxf(x, -125.f);
+  const float shifter = 12582912.f;
+  const float y = x + shifter;
+  const float f = x - (y - shifter);
+  float p = fmaf(0.00132764725f, f, 0.00967554096f);
+  p = fmaf(p, f, 0.0555071309f);
+  p = fmaf(p, f, 0.240221202f);
+  p = fmaf(p, f, 0.693146944f);
+  p = fmaf(p, f, 1.00000012f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(y) << 23));
+}
+
+// ---- packed pairs of fp32 (Blackwell f32x2 arithmetic: one instruction, two lanes of work)
+__device__ __forceinline__ uint64_t f2_pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t r, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// exp2_poly3 on a packed pair (same reduction and polynomial as exp2_poly3);
+// the caller clamps both inputs to >= -125.
+__device__ __forceinline__ void exp2_poly3_x2(uint64_t x2, float& p0, float& p1) {
+  const uint64_t shift = f2_pack(12582912.f, 12582912.f);
+  const uint64_t nshift = f2_pack(-12582912.f, -12582912.f);
+  const uint64_t minus1 = f2_pack(-1.f, -1.f);
+  const uint64_t y = f2_add(x2, shift);
+  const uint64_t f = f2_fma(f2_add(y, nshift), minus1, x2);   // x - round(x)
+  uint64_t p = f2_fma(f2_pack(0.0551716685f, 0.0551716685f), f, f2_pack(0.242611125f, 0.242611125f));
+  p = f2_fma(p, f, f2_pack(0.693260968f, 0.693260968f));
+  p = f2_fma(p, f, f2_pack(0.999928057f, 0.999928057f));
+  float y0, y1;
+  f2_unpack(y, y0, y1);
+  f2_unpack(p, p0, p1);
+  p0 = __int_as_float(__float_as_int(p0) + (__float_as_int(y0) << 23));
+  p1 = __int_as_float(__float_as_int(p1) + (__float_as_int(y1) << 23));
+}
+
+// Register split between warpgroups (all four warps of a warpgroup execute it).
+template <int N>
+__device__ __forceinline__ void regs_release() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_acquire() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);

@@ -24,7 +24,7 @@ def built():
 def header_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(crisp_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(crisp_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_library_exports_every_declared_function():

@@ -248,6 +248,18 @@ def test_tensor_core_and_cuda_core_proxy_agree(base, n, hq, hkv):
         np.testing.assert_allclose(res[0][f], res[1][f], rtol=1e-4, atol=1e-7)
 
 
+def test_fma_pipe_exp2_against_cuda_exp2f():
+    x = torch.cat([torch.linspace(-124.0, 8.0, 1 << 20), torch.tensor([0.0, -0.5, 0.5, -1.0, 7.99, -123.7])]).cuda()
+    p3, p5, ref = crisp.exp2_selftest(x)
+    torch.cuda.synchronize()
+    r = ref.double()
+    e3 = ((p3.double() - r).abs() / r).max().item()
+    e5 = ((p5.double() - r).abs() / r).max().item()
+    # minimax bounds of the fits (7.5e-5 and 2.3e-7) plus exp2f's own error
+    assert e3 < 8e-5, e3
+    assert e5 < 4e-7, e5
+
+
 def test_repeat_calls_are_deterministic():
     layer = S.generate(S.scaled("D", n=2048, h_q=14, h_kv=2))
     q, k, v = device_layer(layer)
