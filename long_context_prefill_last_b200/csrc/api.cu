@@ -32,7 +32,7 @@ WsLayout ws_layout(const Shape& s) {
   L.tile_b = take(hq * nb * 4);
   L.qbar = take(hq * nb * kHeadDim * 4);
   L.kbar = take(hkv * nb * kHeadDim * 4);
-  L.tri = take(hq * (size_t)s.tri * 4);
+  L.tri = take(hq * (size_t)s.tri_stride * 4);
   L.hist = take(hq * sizeof(PeHist));
   L.pe_state = take(hq * sizeof(PeState));
   L.tie_rows = take(hq * nb * 4);
@@ -101,6 +101,7 @@ static crisp_status make_shape(const crisp_cfg* c, Shape* s) {
   s->n_chunks = (s->nb + kChunkTiles - 1) / kChunkTiles;
   s->last_q = c->last_q;
   s->tri = (long long)s->nb * (s->nb + 1) / 2;
+  s->tri_stride = (s->tri + 63) & ~63LL;
   s->fp32 = c->dtype == CRISP_FP32;
   s->sm_scale = c->sm_scale > 0.f ? c->sm_scale : 1.f / sqrtf((float)c->d);
   s->scale_log2 = s->sm_scale * 1.4426950408889634f;

@@ -40,7 +40,8 @@ struct WsLayout {
 
 struct Shape {
   int n, h_q, h_kv, d, group, nb, words, n_chunks, last_q;
-  long long tri;  // entries of the causal block triangle
+  long long tri;         // entries of the causal block triangle
+  long long tri_stride;  // floats reserved per head for it (tri rounded up to 64)
   bool fp32;
   float sm_scale;     // natural-log domain scale
   float scale_log2;   // sm_scale * log2(e)

@@ -18,7 +18,7 @@ namespace {
 
 struct PeArgs {
   int n, nb, words, group, h_q, h_kv;
-  long long tri;
+  long long tri, tri_stride;
   float scale_log2;
   float gamma;
   const int32_t* route;
@@ -37,43 +37,96 @@ struct PeArgs {
 
 __device__ __forceinline__ long long tri_off(int r) { return (long long)r * (r + 1) / 2; }
 
-// Block mean of 128 rows of x[head] -> out[head][b][:] (fp32). One CTA per (block, head).
+__device__ __forceinline__ float warp_max(float v) {
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_min(float v) {
+  for (int o = 16; o > 0; o >>= 1) v = fminf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// 16 bytes of T widened to fp32.
+template <typename T>
+struct Vec16;
+template <>
+struct Vec16<__nv_bfloat16> {
+  static constexpr int N = 8;
+  __device__ static void load(const __nv_bfloat16* p, float (&o)[8]) {
+    const uint4 u = *reinterpret_cast<const uint4*>(p);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      o[2 * i] = __uint_as_float(w[i] << 16);
+      o[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+  }
+};
+template <>
+struct Vec16<float> {
+  static constexpr int N = 4;
+  __device__ static void load(const float* p, float (&o)[4]) {
+    const float4 u = *reinterpret_cast<const float4*>(p);
+    o[0] = u.x;
+    o[1] = u.y;
+    o[2] = u.z;
+    o[3] = u.w;
+  }
+};
+
+// Block mean of 128 rows of x[head] -> out[head][b][:] (fp32). One CTA per
+// (block, head); 16-byte loads, 128 / N threads per row, N rows at a time.
 template <typename T>
 __global__ void __launch_bounds__(128) pool_kernel(const T* __restrict__ x, float* __restrict__ out, int n, int nb,
-                                                   const int32_t* __restrict__ flag, int flag_div) {
+                                                   const int32_t* __restrict__ flag) {
   const int b = blockIdx.x, head = blockIdx.y;
-  if (flag[head / flag_div] == 0) return;   // route check (query heads) or group check (KV heads)
-  __shared__ float red[8][kHeadDim];
-  const int tid = threadIdx.x, rg = tid >> 4, c8 = (tid & 15) * 8;
-  float acc[8];
+  if (flag[head] == 0) return;   // route (query heads) or PE-group flag (KV heads)
+  constexpr int N = Vec16<T>::N;
+  constexpr int TPR = kHeadDim / N;   // threads per row
+  constexpr int RP = 128 / TPR;       // rows in parallel
+  __shared__ float red[RP][kHeadDim];
+  const int tid = threadIdx.x, rg = tid / TPR, c0 = (tid % TPR) * N;
+  float acc[N];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) acc[j] = 0.f;
-  const T* base = x + ((size_t)head * n + (size_t)b * kBlock) * kHeadDim;
-  for (int row = rg; row < kBlock; row += 8) {
-    const T* p = base + (size_t)row * kHeadDim + c8;
+  for (int j = 0; j < N; ++j) acc[j] = 0.f;
+  const T* base = x + ((size_t)head * n + (size_t)b * kBlock) * kHeadDim + c0;
+#pragma unroll 4
+  for (int row = rg; row < kBlock; row += RP) {
+    float v[N];
+    Vec16<T>::load(base + (size_t)row * kHeadDim, v);
 #pragma unroll
-    for (int j = 0; j < 8; ++j) acc[j] += dev::to_f32(p[j]);
+    for (int j = 0; j < N; ++j) acc[j] += v[j];
   }
 #pragma unroll
-  for (int j = 0; j < 8; ++j) red[rg][c8 + j] = acc[j];
+  for (int j = 0; j < N; ++j) red[rg][c0 + j] = acc[j];
   __syncthreads();
   float s = 0.f;
 #pragma unroll
-  for (int g = 0; g < 8; ++g) s += red[g][tid];
+  for (int g = 0; g < RP; ++g) s += red[g][tid];
   out[((size_t)head * nb + b) * kHeadDim + tid] = s * (1.f / kBlock);
 }
 
-// Pooled logits (log2 domain) of 64 query blocks against all key blocks c <= r.
-// Tiles of 64 x 64 outputs; thread (ty, tx) holds a 4 x 4 register tile.
-// Both operand tiles sit transposed in shared memory ([d][block], row stride
-// 68 floats) so one float4 of each feeds 16 FMAs.
+// Pooled logits (log2 domain) of one 64 x 64 tile (rt, ct), ct <= rt, of the
+// block-causal triangle; thread (ty, tx) holds a 4 x 4 register tile. Both
+// operand tiles sit transposed in shared memory ([d][block], row stride 68
+// floats) so one float4 of each feeds 16 FMAs.
 constexpr int kLT = 64;       // blocks per tile side
 constexpr int kLStride = 68;  // floats per transposed row
 __global__ void __launch_bounds__(256) pe_logits_kernel(PeArgs a) {
   const int h = blockIdx.y;
   if (a.route[h] != 1) return;
   const int g = h / a.group;
-  const int r0 = blockIdx.x * kLT;
+  // linear lower-triangle tile index -> (rt, ct)
+  const int ti = blockIdx.x;
+  int rt = (int)((sqrtf(8.f * (float)ti + 1.f) - 1.f) * 0.5f);
+  while ((rt + 1) * (rt + 2) / 2 <= ti) ++rt;
+  while (rt * (rt + 1) / 2 > ti) --rt;
+  const int ct = ti - rt * (rt + 1) / 2;
+  const int r0 = rt * kLT, c0 = ct * kLT;
   extern __shared__ __align__(16) float lsm[];
   float* qT = lsm;                        // [128][kLStride]
   float* kT = lsm + kHeadDim * kLStride;  // [128][kLStride]
@@ -82,42 +135,35 @@ __global__ void __launch_bounds__(256) pe_logits_kernel(PeArgs a) {
     const int rr = e >> 7, dd = e & 127;
     qT[dd * kLStride + rr] =
         (r0 + rr < a.nb) ? a.qbar[((size_t)h * a.nb + r0 + rr) * kHeadDim + dd] * a.scale_log2 : 0.f;
+    kT[dd * kLStride + rr] = (c0 + rr < a.nb) ? a.kbar[((size_t)g * a.nb + c0 + rr) * kHeadDim + dd] : 0.f;
   }
+  __syncthreads();
   const int ty = tid >> 4, tx = tid & 15;
-  const int rmax = min(r0 + kLT - 1, a.nb - 1);
-  for (int c0 = 0; c0 <= rmax; c0 += kLT) {
-    __syncthreads();
-    for (int e = tid; e < kLT * kHeadDim; e += 256) {
-      const int cc = e >> 7, dd = e & 127;
-      kT[dd * kLStride + cc] = (c0 + cc < a.nb) ? a.kbar[((size_t)g * a.nb + c0 + cc) * kHeadDim + dd] : 0.f;
-    }
-    __syncthreads();
-    float acc[4][4];
+  float acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+#pragma unroll 4
+  for (int dd = 0; dd < kHeadDim; ++dd) {
+    const float4 qv = *reinterpret_cast<const float4*>(qT + dd * kLStride + ty * 4);
+    const float4 kv = *reinterpret_cast<const float4*>(kT + dd * kLStride + tx * 4);
+    const float qa[4] = {qv.x, qv.y, qv.z, qv.w};
+    const float ka[4] = {kv.x, kv.y, kv.z, kv.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
-#pragma unroll 4
-    for (int dd = 0; dd < kHeadDim; ++dd) {
-      const float4 qv = *reinterpret_cast<const float4*>(qT + dd * kLStride + ty * 4);
-      const float4 kv = *reinterpret_cast<const float4*>(kT + dd * kLStride + tx * 4);
-      const float qa[4] = {qv.x, qv.y, qv.z, qv.w};
-      const float ka[4] = {kv.x, kv.y, kv.z, kv.w};
+      for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(qa[i], ka[j], acc[i][j]);
+  }
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
+  for (int i = 0; i < 4; ++i) {
+    const int r = r0 + ty * 4 + i;
+    if (r >= a.nb) continue;
+    float* row = a.tri_buf + (size_t)h * a.tri_stride + tri_off(r);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(qa[i], ka[j], acc[i][j]);
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int r = r0 + ty * 4 + i;
-      if (r >= a.nb) continue;
-      float* row = a.tri_buf + (size_t)h * a.tri + tri_off(r);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int c = c0 + tx * 4 + j;
-        if (c <= r) row[c] = acc[i][j];
-      }
+    for (int j = 0; j < 4; ++j) {
+      const int c = c0 + tx * 4 + j;
+      if (c <= r) row[c] = acc[i][j];
     }
   }
 }
@@ -128,84 +174,62 @@ __device__ __forceinline__ void hist_flush(PeHist* hist, uint32_t bucket, unsign
   atomicAdd(&hist->mass[bucket], mass);
 }
 
-__device__ float block_reduce_max(float v, float* sh) {
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  if ((threadIdx.x & 31) == 0) sh[threadIdx.x >> 5] = v;
-  __syncthreads();
-  float r = -INFINITY;
-  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) r = fmaxf(r, sh[w]);
-  __syncthreads();
-  return r;
-}
-__device__ float block_reduce_sum(float v, float* sh) {
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  if ((threadIdx.x & 31) == 0) sh[threadIdx.x >> 5] = v;
-  __syncthreads();
-  float r = 0.f;
-  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) r += sh[w];
-  __syncthreads();
-  return r;
-}
+constexpr int kWin = 64;       // level-0 buckets a row's values may span for the shared-memory path
+constexpr int kRowsPerCta = 8;  // one warp per row
 
-__device__ float block_reduce_min(float v, float* sh) {
-  for (int o = 16; o > 0; o >>= 1) v = fminf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  if ((threadIdx.x & 31) == 0) sh[threadIdx.x >> 5] = v;
-  __syncthreads();
-  float r = INFINITY;
-  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) r = fminf(r, sh[w]);
-  __syncthreads();
-  return r;
-}
-
-constexpr int kWin = 64;   // level-0 buckets a row's values may span for the shared-memory path
-
-// Row softmax of the pooled logits, divided by N_b (the flattened map's total),
-// written in place; level-0 histogram (bits 31..20) with float64 mass. A row's
-// values span few buckets, so counts and mass are first gathered in a
-// shared-memory window and flushed with one global atomic per bucket.
+// Row softmax of the pooled logits, divided by N_b (the flattened map's
+// total), written in place; level-0 histogram (bits 31..20) with float64
+// mass. One warp per row. A row's values span few buckets, so counts and
+// mass gather in a per-warp shared-memory window first and reach the global
+// histogram with one atomic per bucket.
 __global__ void __launch_bounds__(256) pe_softmax_kernel(PeArgs a) {
-  const int h = blockIdx.y, r = blockIdx.x;
+  const int h = blockIdx.y;
   if (a.route[h] != 1) return;
-  __shared__ float sh[32];
-  __shared__ unsigned long long wcount[kWin];
-  __shared__ double wmass[kWin];
-  float* row = a.tri_buf + (size_t)h * a.tri + tri_off(r);
-  float m = -INFINITY, mn = INFINITY;
-  for (int c = threadIdx.x; c <= r; c += blockDim.x) {
-    m = fmaxf(m, row[c]);
-    mn = fminf(mn, row[c]);
+  __shared__ unsigned long long wcount[kRowsPerCta][kWin];
+  __shared__ double wmass[kRowsPerCta][kWin];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = blockIdx.x * kRowsPerCta + warp;
+  for (int i = lane; i < kWin; i += 32) {
+    wcount[warp][i] = 0;
+    wmass[warp][i] = 0.0;
   }
-  m = block_reduce_max(m, sh);
-  mn = block_reduce_min(mn, sh);
+  __syncwarp();
+  if (r >= a.nb) return;
+  float* row = a.tri_buf + (size_t)h * a.tri_stride + tri_off(r);
+  float m = -INFINITY, mn = INFINITY;
+  for (int c = lane; c <= r; c += 32) {
+    const float v = row[c];
+    m = fmaxf(m, v);
+    mn = fminf(mn, v);
+  }
+  m = warp_max(m);
+  mn = warp_min(mn);
   float s = 0.f;
-  for (int c = threadIdx.x; c <= r; c += blockDim.x) s += dev::ex2(row[c] - m);
-  s = block_reduce_sum(s, sh);
+  for (int c = lane; c <= r; c += 32) s += dev::ex2(row[c] - m);
+  s = warp_sum(s);
   const float inv = 1.f / (s * (float)a.nb);
-  const uint32_t b_hi = __float_as_uint(dev::ex2(0.f) * inv) >> 20;      // bucket of the row maximum
+  const uint32_t b_hi = __float_as_uint(inv) >> 20;                       // bucket of the row maximum
   const uint32_t b_lo = __float_as_uint(dev::ex2(mn - m) * inv) >> 20;   // bucket of the row minimum
   const bool window = b_hi >= b_lo && b_hi - b_lo < (uint32_t)kWin;
-  for (int i = threadIdx.x; i < kWin; i += blockDim.x) {
-    wcount[i] = 0;
-    wmass[i] = 0.0;
-  }
-  __syncthreads();
   PeHist* hist = a.hist + h;
   uint32_t cur = 0xffffffffu;
   unsigned long long cnt = 0;
   double mass = 0.0;
-  for (int c = threadIdx.x; c <= r; c += blockDim.x) {
+  auto flush = [&]() {
+    if (!cnt) return;
+    if (window && cur >= b_lo && cur - b_lo < (uint32_t)kWin) {
+      atomicAdd(&wcount[warp][cur - b_lo], cnt);
+      atomicAdd(&wmass[warp][cur - b_lo], mass);
+    } else {
+      hist_flush(hist, cur, cnt, mass);
+    }
+  };
+  for (int c = lane; c <= r; c += 32) {
     const float v = dev::ex2(row[c] - m) * inv;
     row[c] = v;
     const uint32_t bucket = __float_as_uint(v) >> 20;
     if (bucket != cur) {
-      if (cnt) {
-        if (window && cur >= b_lo && cur - b_lo < (uint32_t)kWin) {
-          atomicAdd(&wcount[cur - b_lo], cnt);
-          atomicAdd(&wmass[cur - b_lo], mass);
-        } else {
-          hist_flush(hist, cur, cnt, mass);
-        }
-      }
+      flush();
       cur = bucket;
       cnt = 0;
       mass = 0.0;
@@ -213,23 +237,17 @@ __global__ void __launch_bounds__(256) pe_softmax_kernel(PeArgs a) {
     ++cnt;
     mass += (double)v;
   }
-  if (cnt) {
-    if (window && cur >= b_lo && cur - b_lo < (uint32_t)kWin) {
-      atomicAdd(&wcount[cur - b_lo], cnt);
-      atomicAdd(&wmass[cur - b_lo], mass);
-    } else {
-      hist_flush(hist, cur, cnt, mass);
-    }
-  }
-  __syncthreads();
+  flush();
+  __syncwarp();
   if (window) {
-    for (int i = threadIdx.x; i < kWin; i += blockDim.x)
-      if (wcount[i]) hist_flush(hist, b_lo + i, wcount[i], wmass[i]);
+    for (int i = lane; i < kWin; i += 32)
+      if (wcount[warp][i]) hist_flush(hist, b_lo + i, wcount[warp][i], wmass[warp][i]);
   }
 }
 
 // Histogram of the entries whose key matches the prefix found so far
-// (level 1: bits 19..8 under the 12-bit prefix; level 2: bits 7..0 under the 24-bit prefix).
+// (level 1: bits 19..8 under the 12-bit prefix; level 2: bits 7..0 under the
+// 24-bit prefix). float4 sweeps over the head's triangle (stride padded to 64).
 __global__ void __launch_bounds__(256) pe_hist_kernel(PeArgs a, int level) {
   const int h = blockIdx.y;
   if (a.route[h] != 1) return;
@@ -239,16 +257,21 @@ __global__ void __launch_bounds__(256) pe_hist_kernel(PeArgs a, int level) {
   const int shift_p = level == 1 ? 20 : 8;
   const int shift_b = level == 1 ? 8 : 0;
   const uint32_t bmask = level == 1 ? 0xFFFu : 0xFFu;
-  const float* tri = a.tri_buf + (size_t)h * a.tri;
+  const float4* tri4 = reinterpret_cast<const float4*>(a.tri_buf + (size_t)h * a.tri_stride);
   PeHist* hist = a.hist + h;
-  for (long long p = (long long)blockIdx.x * blockDim.x + threadIdx.x; p < a.tri;
-       p += (long long)gridDim.x * blockDim.x) {
-    const float v = tri[p];
-    const uint32_t key = __float_as_uint(v);
-    if ((key >> shift_p) == prefix) {
-      const uint32_t b = (key >> shift_b) & bmask;
-      atomicAdd(&hist->count[b], 1ull);
-      atomicAdd(&hist->mass[b], (double)v);
+  const long long n4 = (a.tri + 3) / 4;
+  for (long long p = (long long)blockIdx.x * blockDim.x + threadIdx.x; p < n4; p += (long long)gridDim.x * blockDim.x) {
+    const float4 v4 = tri4[p];
+    const float vv[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      if (4 * p + i >= a.tri) break;
+      const uint32_t key = __float_as_uint(vv[i]);
+      if ((key >> shift_p) == prefix) {
+        const uint32_t b = (key >> shift_b) & bmask;
+        atomicAdd(&hist->count[b], 1ull);
+        atomicAdd(&hist->mass[b], (double)vv[i]);
+      }
     }
   }
 }
@@ -364,89 +387,94 @@ __global__ void __launch_bounds__(1024) pe_find_kernel(PeArgs a, int level) {
   }
 }
 
-// Ties needed in part only: count entries equal to the cut value per row.
+// Ties needed in part only: count entries equal to the cut value per row (one warp per row).
 __global__ void __launch_bounds__(256) pe_tie_count_kernel(PeArgs a) {
-  const int h = blockIdx.y, r = blockIdx.x;
+  const int h = blockIdx.y;
   if (a.route[h] != 1) return;
   const PeState* st = a.state + h;
   if (st->all || st->t_keep >= st->n_ties) return;
-  __shared__ float sh[32];
-  const float* row = a.tri_buf + (size_t)h * a.tri + tri_off(r);
-  float cnt = 0.f;
-  for (int c = threadIdx.x; c <= r; c += blockDim.x) cnt += (__float_as_uint(row[c]) == st->cut_key) ? 1.f : 0.f;
-  cnt = block_reduce_sum(cnt, sh);
-  if (threadIdx.x == 0) a.tie_rows[(size_t)h * a.nb + r] = (uint32_t)cnt;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = blockIdx.x * kRowsPerCta + warp;
+  if (r >= a.nb) return;
+  const float* row = a.tri_buf + (size_t)h * a.tri_stride + tri_off(r);
+  uint32_t cnt = 0;
+  for (int c = lane; c <= r; c += 32) cnt += (__float_as_uint(row[c]) == st->cut_key) ? 1u : 0u;
+  for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+  if (lane == 0) a.tie_rows[(size_t)h * a.nb + r] = cnt;
 }
 
-__global__ void __launch_bounds__(32) pe_tie_scan_kernel(PeArgs a) {
+// Exclusive scan of the per-row tie counts (one CTA of 1024 threads per head).
+__global__ void __launch_bounds__(1024) pe_tie_scan_kernel(PeArgs a) {
   const int h = blockIdx.x;
   if (a.route[h] != 1) return;
   const PeState* st = a.state + h;
   if (st->all || st->t_keep >= st->n_ties) return;
-  if (threadIdx.x != 0) return;
-  uint32_t acc = 0;
-  for (int r = 0; r < a.nb; ++r) {
-    const uint32_t v = a.tie_rows[(size_t)h * a.nb + r];
-    a.tie_rows[(size_t)h * a.nb + r] = acc;
+  __shared__ uint32_t part[1024];
+  uint32_t* rows = a.tie_rows + (size_t)h * a.nb;
+  const int per = (a.nb + 1023) / 1024;
+  const int lo = threadIdx.x * per, hi = min(a.nb, lo + per);
+  uint32_t s = 0;
+  for (int r = lo; r < hi; ++r) s += rows[r];
+  part[threadIdx.x] = s;
+  __syncthreads();
+  for (int off = 1; off < 1024; off <<= 1) {
+    const uint32_t v = threadIdx.x >= off ? part[threadIdx.x - off] : 0u;
+    __syncthreads();
+    part[threadIdx.x] += v;
+    __syncthreads();
+  }
+  uint32_t acc = threadIdx.x > 0 ? part[threadIdx.x - 1] : 0u;
+  for (int r = lo; r < hi; ++r) {
+    const uint32_t v = rows[r];
+    rows[r] = acc;
     acc += v;
   }
 }
 
-// Write the PE mask row by row: keep (r, c), c <= r, when its value is above
-// the cut, or equal to it and among the first t_keep ties in flat order, or
-// c == r; or everything when the cut keeps all.
+// Write the PE mask row by row (one warp per row): keep (r, c), c <= r, when
+// its value is above the cut, or equal to it and among the first t_keep ties
+// in flat order, or c == r; or everything when the cut keeps all.
 __global__ void __launch_bounds__(256) pe_mask_kernel(PeArgs a) {
-  const int h = blockIdx.y, r = blockIdx.x;
+  const int h = blockIdx.y;
   if (a.route[h] != 1) return;
   const PeState* st = a.state + h;
-  __shared__ int warp_sums[9];
-  __shared__ float shr[32];
-  const bool all = st->all != 0;
-  const uint32_t cut = st->cut_key;
-  const bool partial_ties = !all && st->t_keep < st->n_ties;
-  const unsigned long long t_keep = st->t_keep;
-  unsigned long long tie_base = partial_ties ? a.tie_rows[(size_t)h * a.nb + r] : 0ull;
-  const float* row = a.tri_buf + (size_t)h * a.tri + tri_off(r);
-  uint32_t* mrow = a.pe_mask + ((size_t)h * a.nb + r) * a.words;
-  float kept = 0.f;
-  for (int c0 = 0; c0 < a.words * 32; c0 += blockDim.x) {
-    const int c = c0 + threadIdx.x;
-    int keep = 0, tie = 0;
-    if (c <= r) {
-      const uint32_t key = __float_as_uint(row[c]);
-      tie = (!all && key == cut) ? 1 : 0;
-      keep = all || c == r || key > cut || (tie && !partial_ties);
-    }
-    if (partial_ties) {
-      // rank of this tie among the ties of the head in flat order
-      const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-      const unsigned bal = __ballot_sync(0xffffffffu, tie);
-      if (lane == 0) warp_sums[wid] = __popc(bal);
-      __syncthreads();
-      if (threadIdx.x == 0) {
-        int acc = 0;
-        for (int w = 0; w < 8; ++w) {
-          const int v = warp_sums[w];
-          warp_sums[w] = acc;
-          acc += v;
-        }
-        warp_sums[8] = acc;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = blockIdx.x * kRowsPerCta + warp;
+  __shared__ unsigned long long kept_cta;
+  if (threadIdx.x == 0) kept_cta = 0;
+  __syncthreads();
+  if (r < a.nb) {
+    const bool all = st->all != 0;
+    const uint32_t cut = st->cut_key;
+    const bool partial_ties = !all && st->t_keep < st->n_ties;
+    const unsigned long long t_keep = st->t_keep;
+    unsigned long long tie_base = partial_ties ? a.tie_rows[(size_t)h * a.nb + r] : 0ull;
+    const float* row = a.tri_buf + (size_t)h * a.tri_stride + tri_off(r);
+    uint32_t* mrow = a.pe_mask + ((size_t)h * a.nb + r) * a.words;
+    uint32_t kept = 0;
+    for (int w = 0; w < a.words; ++w) {
+      const int c = w * 32 + lane;
+      int keep = 0, tie = 0;
+      if (c <= r) {
+        const uint32_t key = __float_as_uint(row[c]);
+        tie = (!all && key == cut) ? 1 : 0;
+        keep = all || c == r || key > cut || (tie && !partial_ties);
       }
-      __syncthreads();
-      const unsigned long long rank = tie_base + warp_sums[wid] + __popc(bal & ((1u << lane) - 1u));
-      if (tie && rank < t_keep) keep = 1;
-      tie_base += warp_sums[8];
-      __syncthreads();
+      if (partial_ties) {
+        const unsigned tb = __ballot_sync(0xffffffffu, tie);
+        const unsigned long long rank = tie_base + __popc(tb & ((1u << lane) - 1u));
+        if (tie && rank < t_keep) keep = 1;
+        tie_base += __popc(tb);
+      }
+      const unsigned bal = __ballot_sync(0xffffffffu, keep);
+      if (lane == 0) mrow[w] = bal;
+      kept += __popc(bal);
     }
-    const unsigned bal = __ballot_sync(0xffffffffu, keep);
-    if ((threadIdx.x & 31) == 0 && (c >> 5) < a.words) mrow[c >> 5] = bal;
-    kept += keep ? 1.f : 0.f;
+    if (lane == 0) atomicAdd(&kept_cta, (unsigned long long)kept);
+    if (lane == 0 && r == 0) a.pe_cut[h] = all ? 0.f : __uint_as_float(cut);
   }
-  kept = block_reduce_sum(kept, shr);
-  if (threadIdx.x == 0) {
-    atomicAdd(reinterpret_cast<unsigned long long*>(a.pe_count + h), (unsigned long long)kept);
-    if (r == 0) a.pe_cut[h] = all ? 0.f : __uint_as_float(cut);
-  }
+  __syncthreads();
+  if (threadIdx.x == 0 && kept_cta) atomicAdd(reinterpret_cast<unsigned long long*>(a.pe_count + h), kept_cta);
 }
 
 }  // namespace
@@ -461,6 +489,7 @@ cudaError_t launch_pe(const void* q, const void* k, const Shape& s, char* ws, co
   a.h_q = s.h_q;
   a.h_kv = s.h_kv;
   a.tri = s.tri;
+  a.tri_stride = s.tri_stride;
   a.scale_log2 = s.scale_log2;
   a.gamma = s.gamma;
   a.route = ix.route;
@@ -478,33 +507,33 @@ cudaError_t launch_pe(const void* q, const void* k, const Shape& s, char* ws, co
 
   cudaError_t e = cudaMemsetAsync(a.hist, 0, sizeof(PeHist) * s.h_q, st);
   if (e != cudaSuccess) return e;
-  // the query-head pooling is gated by the route; the key pooling by kv_pe
-  // (route values 1 = PE are used directly as the flag).
+  // the query-head pooling is gated by the route (1 = PE); the key pooling
+  // by the per-group PE flag
   if (s.fp32) {
-    pool_kernel<float><<<dim3(s.nb, s.h_q), 128, 0, st>>>(static_cast<const float*>(q), a.qbar, s.n, s.nb,
-                                                          ix.route, 1);
-    pool_kernel<float><<<dim3(s.nb, s.h_kv), 128, 0, st>>>(static_cast<const float*>(k), a.kbar, s.n, s.nb,
-                                                           a.kv_pe, 1);
+    pool_kernel<float><<<dim3(s.nb, s.h_q), 128, 0, st>>>(static_cast<const float*>(q), a.qbar, s.n, s.nb, ix.route);
+    pool_kernel<float><<<dim3(s.nb, s.h_kv), 128, 0, st>>>(static_cast<const float*>(k), a.kbar, s.n, s.nb, a.kv_pe);
   } else {
     pool_kernel<__nv_bfloat16><<<dim3(s.nb, s.h_q), 128, 0, st>>>(static_cast<const __nv_bfloat16*>(q), a.qbar,
-                                                                  s.n, s.nb, ix.route, 1);
+                                                                  s.n, s.nb, ix.route);
     pool_kernel<__nv_bfloat16><<<dim3(s.nb, s.h_kv), 128, 0, st>>>(static_cast<const __nv_bfloat16*>(k), a.kbar,
-                                                                   s.n, s.nb, a.kv_pe, 1);
+                                                                   s.n, s.nb, a.kv_pe);
   }
   const size_t lsmem = 2 * kHeadDim * kLStride * sizeof(float);
   e = cudaFuncSetAttribute(pe_logits_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lsmem);
   if (e != cudaSuccess) return e;
-  pe_logits_kernel<<<dim3((s.nb + kLT - 1) / kLT, s.h_q), 256, lsmem, st>>>(a);
-  pe_softmax_kernel<<<dim3(s.nb, s.h_q), 256, 0, st>>>(a);
+  const int nt = (s.nb + kLT - 1) / kLT;
+  pe_logits_kernel<<<dim3(nt * (nt + 1) / 2, s.h_q), 256, lsmem, st>>>(a);
+  const int row_ctas = (s.nb + kRowsPerCta - 1) / kRowsPerCta;
+  pe_softmax_kernel<<<dim3(row_ctas, s.h_q), 256, 0, st>>>(a);
   pe_find_kernel<<<s.h_q, 1024, 0, st>>>(a, 0);
-  const int hist_ctas = (int)std::min<long long>(1184, (s.tri + 255) / 256);
+  const int hist_ctas = (int)std::min<long long>(1184, (s.tri / 4 + 255) / 256 + 1);
   pe_hist_kernel<<<dim3(hist_ctas, s.h_q), 256, 0, st>>>(a, 1);
   pe_find_kernel<<<s.h_q, 1024, 0, st>>>(a, 1);
   pe_hist_kernel<<<dim3(hist_ctas, s.h_q), 256, 0, st>>>(a, 2);
   pe_find_kernel<<<s.h_q, 1024, 0, st>>>(a, 2);
-  pe_tie_count_kernel<<<dim3(s.nb, s.h_q), 256, 0, st>>>(a);
-  pe_tie_scan_kernel<<<s.h_q, 32, 0, st>>>(a);
-  pe_mask_kernel<<<dim3(s.nb, s.h_q), 256, 0, st>>>(a);
+  pe_tie_count_kernel<<<dim3(row_ctas, s.h_q), 256, 0, st>>>(a);
+  pe_tie_scan_kernel<<<s.h_q, 1024, 0, st>>>(a);
+  pe_mask_kernel<<<dim3(row_ctas, s.h_q), 256, 0, st>>>(a);
   return cudaGetLastError();
 }
 

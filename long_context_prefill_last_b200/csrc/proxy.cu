@@ -153,18 +153,22 @@ __global__ void __launch_bounds__(256) proxy_simt_kernel(const T* __restrict__ q
 
 // Row normalisers: M_i = max over chunks, L_i = sum l * 2^(m - M); chunk
 // weight 2^(m - M) / (L_i * |Q-hat|) turns stored partials into column means.
-__global__ void proxy_row_weights_kernel(const float2* __restrict__ ml, float* __restrict__ w, int n_chunks,
-                                         int32_t* status) {
-  const int h = blockIdx.x, r = threadIdx.x;
-  const size_t row = (size_t)h * kProxyRows + r;
-  const float2* p = ml + row * n_chunks;
+// One warp per proxy row, lanes over chunks.
+__global__ void __launch_bounds__(256) proxy_row_weights_kernel(const float2* __restrict__ ml, float* __restrict__ w,
+                                                                int rows, int n_chunks, int32_t* status) {
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const float2* p = ml + (size_t)row * n_chunks;
   float M = -INFINITY;
-  for (int c = 0; c < n_chunks; ++c) M = fmaxf(M, p[c].x);
+  for (int c = lane; c < n_chunks; c += 32) M = fmaxf(M, p[c].x);
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
   float L = 0.f;
-  for (int c = 0; c < n_chunks; ++c) L += p[c].y * dev::ex2(p[c].x - M);
-  if (!(L > 0.f) || !isfinite(L) || !isfinite(M)) dev::report(status, CRISP_ERR_NONFINITE, h);
+  for (int c = lane; c < n_chunks; c += 32) L += p[c].y * dev::ex2(p[c].x - M);
+  for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+  if (lane == 0 && (!(L > 0.f) || !isfinite(L) || !isfinite(M)))
+    dev::report(status, CRISP_ERR_NONFINITE, row / kProxyRows);
   const float inv = 1.f / (L * (float)kProxyRows);
-  for (int c = 0; c < n_chunks; ++c) w[row * n_chunks + c] = dev::ex2(p[c].x - M) * inv;
+  for (int c = lane; c < n_chunks; c += 32) w[(size_t)row * n_chunks + c] = dev::ex2(p[c].x - M) * inv;
 }
 
 // Column-block masses p_v[t] and the two diagonal halves of every tile.
@@ -213,7 +217,8 @@ cudaError_t launch_finalize(const Shape& s, char* ws, const WsLayout& L, const I
   const float2* ml = reinterpret_cast<const float2*>(ws + L.chunk_ml);
   float* w = reinterpret_cast<float*>(ws + L.chunk_w);
   int32_t* status = reinterpret_cast<int32_t*>(ws + L.status);
-  proxy_row_weights_kernel<<<s.h_q, kProxyRows, 0, st>>>(ml, w, s.n_chunks, status);
+  const int rows = s.h_q * kProxyRows;
+  proxy_row_weights_kernel<<<(rows + 7) / 8, 256, 0, st>>>(ml, w, rows, s.n_chunks, status);
   dim3 grid((s.nb + 127) / 128, s.h_q);
   proxy_tile_sums_kernel<<<grid, 128, 0, st>>>(reinterpret_cast<const float*>(ws + L.part_lo),
                                                reinterpret_cast<const float*>(ws + L.part_hi), w, ix.p_v,
