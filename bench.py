@@ -241,7 +241,7 @@ def run_crisp(args, rank, world, local_rank):
     out = torch.empty_like(q)
     out_h = torch.empty(q.shape, dtype=q.dtype).pin_memory()
     dtype = crisp.FP32 if c.dtype == "fp32" else crisp.BF16
-    cfg = crisp.Config(n=c.n, h_q=c.h_q, h_kv=c.h_kv, d=c.d, dtype=dtype)
+    cfg = crisp.Config(n=c.n, h_q=c.h_q, h_kv=c.h_kv, d=c.d, dtype=dtype, alpha=args.alpha, gamma=args.gamma)
     cfg.allocate_workspace(dev)
     ix = crisp.IndexBuffers(cfg, dev)
     stream = torch.cuda.current_stream(dev)
@@ -379,6 +379,7 @@ def run_crisp(args, rank, world, local_rank):
         "dtype": "bf16" if c.dtype == "bf16" else "f32",
         "data": "synthetic (seeded Gaussian heads with planted sink/vertical/slash structure; no datasets or weights)",
         "config": {"workload": f"layer {args.config}: {c.desc}", "h_q": c.h_q, "h_kv": c.h_kv, "seq_len": c.n,
+                   "alpha": args.alpha, "gamma": args.gamma,
                    "head_dim": c.d, "batch": 1, "parallelism": f"independent layer per GPU x{world}",
                    "l2": "inputs (>= 6 GiB at 512K) far exceed the 126 MB L2; no flush between steps"},
         "speedup_vs_dense": round(dense_m / step_m, 4),
@@ -421,7 +422,8 @@ def run_stage(args):
     layer = S.generate(c, threads=min(32, os.cpu_count() or 8))
     q, k, v = (t.cuda() for t in S.to_torch(layer))
     out = torch.empty_like(q)
-    cfg = crisp.Config(n=c.n, h_q=c.h_q, h_kv=c.h_kv, dtype=crisp.FP32 if c.dtype == "fp32" else crisp.BF16)
+    cfg = crisp.Config(n=c.n, h_q=c.h_q, h_kv=c.h_kv, dtype=crisp.FP32 if c.dtype == "fp32" else crisp.BF16,
+                       alpha=args.alpha, gamma=args.gamma)
     cfg.allocate_workspace()
     ix = crisp.IndexBuffers(cfg)
     crisp.select(q, k, cfg, ix)
@@ -455,6 +457,8 @@ def main():
     ap.add_argument("--config", default="E", choices=sorted(S.CONFIGS))
     ap.add_argument("--impl", default="crisp", choices=["crisp", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--alpha", type=float, default=1.0, help="Eq. (4) noise-floor multiplier")
+    ap.add_argument("--gamma", type=float, default=0.95, help="PE cumulative coverage")
     ap.add_argument("--only", choices=["select", "attend", "dense", "prefill", "route"],
                     help="profiling mode: time one stage alone (no contract line)")
     ap.add_argument("--n", type=int, help="profiling mode: scaled sequence length")

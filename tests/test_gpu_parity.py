@@ -153,6 +153,8 @@ SMALL = {
     "B-512-min": (lambda: S.scaled("B", n=512, h_q=4, h_kv=1, planted_groups=[0]), {}),
     "B-4224-33blocks": (lambda: S.scaled("B", n=4224, h_q=4, h_kv=2), {}),
     "B-4k-alpha1.5": (lambda: S.scaled("B", n=4096, h_q=8, h_kv=2), {"alpha": 1.5}),
+    "B-4k-alpha1.25-gamma0.97": (lambda: S.scaled("B", n=4096, h_q=8, h_kv=2), {"alpha": 1.25, "gamma": 0.97}),
+    "D-2k-alpha1.5-gamma0.97": (lambda: S.scaled("D", n=2048, h_q=14, h_kv=2), {"alpha": 1.5, "gamma": 0.97}),
     "B-4k-alpha0": (lambda: S.scaled("B", n=4096, h_q=8, h_kv=2), {"alpha": 0.0}),
     "B-4k-gamma1": (lambda: S.scaled("B", n=4096, h_q=8, h_kv=2), {"gamma": 1.0}),
     "B-4k-gamma0.5": (lambda: S.scaled("B", n=4096, h_q=8, h_kv=2), {"gamma": 0.5}),
