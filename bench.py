@@ -377,7 +377,9 @@ def run_crisp(args, rank, world, local_rank):
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "bf16" if c.dtype == "bf16" else "f32",
-        "data": "synthetic (seeded Gaussian heads with planted sink/vertical/slash structure; no datasets or weights)",
+        "data": ("synthetic (seeded Gaussian heads with planted sink/vertical/slash structure"
+                 + (f", log-normal block background sigma {c.cliff_sigma:g}" if c.cliff_sigma > 0 else "")
+                 + "; no datasets or weights)"),
         "config": {"workload": f"layer {args.config}: {c.desc}", "h_q": c.h_q, "h_kv": c.h_kv, "seq_len": c.n,
                    "alpha": args.alpha, "gamma": args.gamma,
                    "head_dim": c.d, "batch": 1, "parallelism": f"independent layer per GPU x{world}",

@@ -44,6 +44,18 @@ Recipe (all randomness from numpy PCG64 seeded by
 * The sink strength for the bf16 layers is set so the sink carries a fraction
   f of a row's mass against the Gaussian background:
   ``sink_logits = ln(f/(1-f)) + ln(n-1) + 1/2``.
+* Mass-cliff background (``cliff_sigma`` > 0): the pages' premise is that
+  real attention mass falls off a cliff, a few blocks holding most of it
+  (summary page, "Theoretical Basis"), which an iid Gaussian background
+  lacks. Every KV group then draws a per-key-block logit offset
+  ``beta_b = cliff_sigma * z_b`` (z_b ~ N(0, 1), seeded per group) for the
+  blocks 1 .. N_b-2; the sink block and the last block keep beta = 0. It
+  is planted like the sink: along u in planted groups, along a seeded unit
+  vector w (Q and K noise projected off w, every query ``+a*w``) in the
+  other groups, so every key of block b gains exactly beta_b logits against
+  every query of the group. Block masses are then log-normal with
+  log-standard-deviation cliff_sigma. The sink logits add ``cliff_sigma**2/2``
+  (the background's mean mass factor) to keep the sink's share.
 """
 from __future__ import annotations
 
@@ -57,7 +69,7 @@ import numpy as np
 BLOCK = 128
 
 # tensor ids for the seed sequence
-_T_Q, _T_K, _T_V, _T_STRUCT, _T_CODES = 0, 1, 2, 3, 4
+_T_Q, _T_K, _T_V, _T_STRUCT, _T_CODES, _T_CLIFF = 0, 1, 2, 3, 4, 5
 
 
 @dataclasses.dataclass(frozen=True)
@@ -76,6 +88,7 @@ class LayerConfig:
     gauss_q_scale: float = 1.0      # Q multiplier on Gaussian groups
     desc: str = ""
     slash_groups: int = 0           # groups the layer's slashes are dealt over (0: planted count)
+    cliff_sigma: float = 0.0        # log-normal block background (0: iid Gaussian background)
 
     @property
     def n_blocks(self) -> int:
@@ -86,14 +99,15 @@ class LayerConfig:
         return self.h_q // self.h_kv
 
 
-def sink_logits_for_fraction(f: float, n: int) -> float:
-    """Extra sink logits so the sink holds fraction f of a Gaussian row's mass."""
-    return math.log(f / (1.0 - f)) + math.log(n - 1) + 0.5
+def sink_logits_for_fraction(f: float, n: int, cliff_sigma: float = 0.0) -> float:
+    """Extra sink logits so the sink holds fraction f of a Gaussian row's mass
+    (with a log-normal block background of log-sd cliff_sigma when given)."""
+    return math.log(f / (1.0 - f)) + math.log(n - 1) + 0.5 + 0.5 * cliff_sigma ** 2
 
 
-def _llama(name, cid, n, n_vert, n_slash, desc):
+def _llama(name, cid, n, n_vert, n_slash, desc, cliff_sigma=0.0):
     return LayerConfig(name, cid, 32, 8, n, 128, "bf16", tuple(range(6)), n_vert, n_slash,
-                       sink_logits_for_fraction(0.5, n), 1.0, desc)
+                       sink_logits_for_fraction(0.5, n, cliff_sigma), 1.0, desc, cliff_sigma=cliff_sigma)
 
 
 CONFIGS: Dict[str, LayerConfig] = {
@@ -105,6 +119,13 @@ CONFIGS: Dict[str, LayerConfig] = {
                      sink_logits_for_fraction(0.9, 131072), 2.0,
                      "Qwen2.5-7B-shaped 28Q/4KV, n=131072, bf16, half VS (sink 90%), half T=0.5"),
     "E": _llama("E", 4, 524288, 128, 32, "Llama-3.1-8B-shaped 32Q/8KV, n=524288, bf16"),
+    # mass-cliff background (log-normal block masses, log-sd 2) on the shapes of C and E
+    "C_cliff": _llama("C_cliff", 5, 131072, 64, 16,
+                      "Llama-3.1-8B-shaped 32Q/8KV, n=131072, bf16, log-normal block background (sigma 2)",
+                      cliff_sigma=2.0),
+    "E_cliff": _llama("E_cliff", 6, 524288, 128, 32,
+                      "Llama-3.1-8B-shaped 32Q/8KV, n=524288, bf16, log-normal block background (sigma 2)",
+                      cliff_sigma=2.0),
 }
 
 
@@ -127,7 +148,7 @@ def scaled(base: str, *, n: Optional[int] = None, h_q: Optional[int] = None,
     sink = c.sink_logits
     if c.dtype == "bf16":
         f = 0.9 if base == "D" else 0.5
-        sink = sink_logits_for_fraction(f, n2)
+        sink = sink_logits_for_fraction(f, n2, c.cliff_sigma)
     nb = -(-n2 // BLOCK)
     # keep the density of verticals per block of the full-size layer
     nv = n_vert if n_vert is not None else min(max(1, round(c.n_vert * n2 / c.n)), max(nb - 2, 0))
@@ -206,6 +227,25 @@ def position_codes(cfg: LayerConfig, g: int, count: int) -> np.ndarray:
     return c
 
 
+def cliff_offsets(cfg: LayerConfig, g: int):
+    """Seeded (w, beta) of KV group g's mass-cliff background: w a unit
+    direction (used by groups without planted structure), beta [N_b] the
+    per-key-block logit offsets (zero for the first and last block)."""
+    r = _rng(cfg, g, _T_CLIFF)
+    w = r.standard_normal(cfg.d)
+    w /= np.linalg.norm(w)
+    nb = cfg.n_blocks
+    beta = cfg.cliff_sigma * r.standard_normal(nb)
+    beta[0] = 0.0
+    beta[nb - 1] = 0.0
+    return w, beta
+
+
+def _key_offsets(cfg: LayerConfig, beta: np.ndarray) -> np.ndarray:
+    """Per-key logit offset: beta of the key's block."""
+    return np.repeat(beta, BLOCK)[: cfg.n]
+
+
 def _project_off(x: np.ndarray, u: np.ndarray) -> None:
     x -= np.outer(x @ u, u).astype(x.dtype)
 
@@ -213,14 +253,22 @@ def _project_off(x: np.ndarray, u: np.ndarray) -> None:
 def _gen_k(cfg: LayerConfig, g: int, st: Optional[GroupStructure]) -> np.ndarray:
     n, d = cfg.n, cfg.d
     k = _rng(cfg, g, _T_K).standard_normal((n, d), dtype=np.float32)
-    if st is None:
-        return k
     a = d ** 0.25
+    if st is None:
+        if cfg.cliff_sigma > 0:
+            w, beta = cliff_offsets(cfg, g)
+            w32 = w.astype(np.float32)
+            _project_off(k, w32)
+            k += (a * _key_offsets(cfg, beta))[:, None].astype(np.float32) * w32[None, :]
+        return k
     k[:, : slash_dims(d)] = 0.0
     _project_off(k, st.u.astype(np.float32))
     # sink: +sink_logits against every query of the group
     k[0] += (cfg.sink_logits * math.sqrt(d) / a * st.u).astype(np.float32)
     k[st.verticals] += (4.0 * a * st.u).astype(np.float32)
+    if cfg.cliff_sigma > 0:
+        _, beta = cliff_offsets(cfg, g)
+        k += (a * _key_offsets(cfg, beta))[:, None].astype(np.float32) * st.u.astype(np.float32)[None, :]
     if len(st.slash_offsets):
         s = np.float32(math.sqrt(4.0 * math.sqrt(d)))
         codes = position_codes(cfg, st.group, n + int(st.slash_offsets.max()))
@@ -234,6 +282,11 @@ def _gen_q(cfg: LayerConfig, h: int, st: Optional[GroupStructure]) -> np.ndarray
     n, d = cfg.n, cfg.d
     q = _rng(cfg, 1000 + h, _T_Q).standard_normal((n, d), dtype=np.float32)
     if st is None:
+        if cfg.cliff_sigma > 0:
+            w, _ = cliff_offsets(cfg, h // cfg.group)
+            w32 = w.astype(np.float32)
+            _project_off(q, w32)
+            q += (d ** 0.25 * w32)[None, :]
         if cfg.gauss_q_scale != 1.0:
             q *= np.float32(cfg.gauss_q_scale)
         return q

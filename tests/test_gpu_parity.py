@@ -160,6 +160,10 @@ SMALL = {
     "B-4k-gamma0.5": (lambda: S.scaled("B", n=4096, h_q=8, h_kv=2), {"gamma": 0.5}),
     "B-4k-forcePE": (lambda: S.scaled("B", n=4096, h_q=8, h_kv=2), {"force_route": 1}),
     "B-4k-alphaHuge": (lambda: S.scaled("B", n=4096, h_q=8, h_kv=2), {"alpha": 1e30}),
+    # mass-cliff background (log-normal block masses): sparser VS and PE selections
+    "Ccliff-4k": (lambda: S.scaled("C_cliff", n=4096, h_q=8, h_kv=2), {}),
+    "Ccliff-16k": (lambda: S.scaled("C_cliff", n=16384, h_q=8, h_kv=2), {}),
+    "Ccliff-4k-alpha1.5-gamma0.97": (lambda: S.scaled("C_cliff", n=4096, h_q=8, h_kv=2), {"alpha": 1.5, "gamma": 0.97}),
 }
 
 
@@ -275,7 +279,7 @@ def test_repeat_calls_are_deterministic():
 
 # ----------------------------------------------------------------------------- full-size layers
 
-@pytest.mark.parametrize("name", ["B", "C", "D", "E"])
+@pytest.mark.parametrize("name", ["B", "C", "D", "E", "E_cliff"])
 def test_full_size_layer_parity(name):
     layer = S.generate(S.CONFIGS[name], threads=16)
     q, k, v = device_layer(layer)
@@ -286,8 +290,14 @@ def test_full_size_layer_parity(name):
     rep = P.Report()
     check_index(host, oidx, cfg, rep)
     rep.assert_ok()
+    if layer.cfg.cliff_sigma > 0:
+        # a cliffed background hides planted keys that sit in light blocks; the
+        # sink still routes planted heads VS and the cliff keeps the selections sparse
+        for h in layer.planted_q_heads:
+            assert host["route"][h] == O.VS
+            assert host["sel_v"][h].mean() < 0.5 and host["sel_s"][h].mean() < 0.5
     # planted structure must be selected, Gaussian heads must route PE
-    for h in layer.planted_q_heads:
+    for h in ([] if layer.cfg.cliff_sigma > 0 else layer.planted_q_heads):
         assert host["route"][h] == O.VS
         st = layer.structure[h // layer.cfg.group]
         assert host["sel_v"][h][st.verticals // 128].all()

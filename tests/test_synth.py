@@ -1,4 +1,5 @@
 """The seeded input generator: determinism, dtype handling and planted geometry."""
+import dataclasses
 import math
 
 import numpy as np
@@ -55,3 +56,36 @@ def test_sink_fraction_formula():
         w_sink = math.exp(dl)
         rest = (n - 1) * math.exp(0.5)
         assert abs(w_sink / (w_sink + rest) - f) < 1e-12
+
+
+def test_cliff_background_offsets_are_exact_per_block():
+    # float32 layer (before any bf16 rounding): every key of block b carries
+    # exactly beta_b extra logits along the group's cliff direction
+    cfg = dataclasses.replace(S.scaled("C_cliff", n=2048, h_q=4, h_kv=2), dtype="fp32")
+    layer = S.generate(cfg, with_v=False)
+    d, a = cfg.d, cfg.d ** 0.25
+    for g in range(cfg.h_kv):
+        w, beta = S.cliff_offsets(cfg, g)
+        assert beta[0] == 0.0 and beta[-1] == 0.0
+        assert abs(np.std(beta[1:-1]) - cfg.cliff_sigma) < 0.5
+        k = layer.k[g].astype(np.float64)
+        q = layer.q[g * cfg.group].astype(np.float64)
+        direction = layer.structure[g].u if g in layer.structure else w
+        # queries: component a along the direction; keys: beta_b * a (sink key 0 aside)
+        assert np.allclose(q @ direction, a, atol=1e-4)
+        kk = k[1:] @ direction
+        expect = a * np.repeat(beta, S.BLOCK)[1:cfg.n]
+        if g in layer.structure:
+            vert = np.zeros(cfg.n, bool)
+            vert[layer.structure[g].verticals] = True
+            expect = expect + np.where(vert[1:], 4 * a, 0.0)
+        assert np.allclose(kk, expect, atol=1e-3)
+
+
+def test_cliff_sink_fraction_formula():
+    # with log-normal block offsets of log-sd sigma the background's mean mass grows by e^(sigma^2/2)
+    f, n, sig = 0.5, 131072, 2.0
+    dl = S.sink_logits_for_fraction(f, n, sig)
+    w_sink = math.exp(dl)
+    rest = (n - 1) * math.exp(0.5) * math.exp(sig * sig / 2)
+    assert abs(w_sink / (w_sink + rest) - f) < 1e-12
