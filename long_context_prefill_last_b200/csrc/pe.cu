@@ -41,10 +41,6 @@ __device__ __forceinline__ float warp_max(float v) {
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
   return v;
 }
-__device__ __forceinline__ float warp_min(float v) {
-  for (int o = 16; o > 0; o >>= 1) v = fminf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
-}
 __device__ __forceinline__ float warp_sum(float v) {
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
@@ -174,91 +170,95 @@ __device__ __forceinline__ void hist_flush(PeHist* hist, uint32_t bucket, unsign
   atomicAdd(&hist->mass[bucket], mass);
 }
 
-constexpr int kWin = 64;       // level-0 buckets a row's values may span for the shared-memory path
 constexpr int kRowsPerCta = 8;  // one warp per row
+// Level-0 buckets (bits 31..20) of the values in [0, 1): every entry of the
+// normalised map is at most 1 / N_b, so its bucket is below 0x3F8.
+constexpr int kL0Low = 1024;
 
 // Row softmax of the pooled logits, divided by N_b (the flattened map's
 // total), written in place; level-0 histogram (bits 31..20) with float64
-// mass. One warp per row. A row's values span few buckets, so counts and
-// mass gather in a per-warp shared-memory window first and reach the global
-// histogram with one atomic per bucket.
+// mass. One warp per row. Each lane merges runs of equal buckets, the CTA
+// gathers counts and mass in a shared-memory histogram of all level-0
+// buckets below 1.0, and the non-empty buckets reach the global histogram
+// with one atomic each.
 __global__ void __launch_bounds__(256) pe_softmax_kernel(PeArgs a) {
   const int h = blockIdx.y;
-  if (a.route[h] != 1) return;
-  __shared__ unsigned long long wcount[kRowsPerCta][kWin];
-  __shared__ double wmass[kRowsPerCta][kWin];
+  if (a.route[h] != 1) return;   // uniform over the CTA
+  __shared__ unsigned long long scount[kL0Low];
+  __shared__ double smass[kL0Low];
+  for (int i = threadIdx.x; i < kL0Low; i += blockDim.x) {
+    scount[i] = 0;
+    smass[i] = 0.0;
+  }
+  __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r = blockIdx.x * kRowsPerCta + warp;
-  for (int i = lane; i < kWin; i += 32) {
-    wcount[warp][i] = 0;
-    wmass[warp][i] = 0.0;
-  }
-  __syncwarp();
-  if (r >= a.nb) return;
-  float* row = a.tri_buf + (size_t)h * a.tri_stride + tri_off(r);
-  float m = -INFINITY, mn = INFINITY;
-  for (int c = lane; c <= r; c += 32) {
-    const float v = row[c];
-    m = fmaxf(m, v);
-    mn = fminf(mn, v);
-  }
-  m = warp_max(m);
-  mn = warp_min(mn);
-  float s = 0.f;
-  for (int c = lane; c <= r; c += 32) s += dev::ex2(row[c] - m);
-  s = warp_sum(s);
-  const float inv = 1.f / (s * (float)a.nb);
-  const uint32_t b_hi = __float_as_uint(inv) >> 20;                       // bucket of the row maximum
-  const uint32_t b_lo = __float_as_uint(dev::ex2(mn - m) * inv) >> 20;   // bucket of the row minimum
-  const bool window = b_hi >= b_lo && b_hi - b_lo < (uint32_t)kWin;
   PeHist* hist = a.hist + h;
-  uint32_t cur = 0xffffffffu;
-  unsigned long long cnt = 0;
-  double mass = 0.0;
-  auto flush = [&]() {
-    if (!cnt) return;
-    if (window && cur >= b_lo && cur - b_lo < (uint32_t)kWin) {
-      atomicAdd(&wcount[warp][cur - b_lo], cnt);
-      atomicAdd(&wmass[warp][cur - b_lo], mass);
-    } else {
-      hist_flush(hist, cur, cnt, mass);
+  if (r < a.nb) {
+    float* row = a.tri_buf + (size_t)h * a.tri_stride + tri_off(r);
+    float m = -INFINITY;
+    for (int c = lane; c <= r; c += 32) m = fmaxf(m, row[c]);
+    m = warp_max(m);
+    float s = 0.f;
+    for (int c = lane; c <= r; c += 32) s += dev::ex2(row[c] - m);
+    s = warp_sum(s);
+    const float inv = 1.f / (s * (float)a.nb);
+    uint32_t cur = 0xffffffffu;
+    unsigned long long cnt = 0;
+    double mass = 0.0;
+    auto flush = [&]() {
+      if (!cnt) return;
+      if (cur < (uint32_t)kL0Low) {
+        atomicAdd(&scount[cur], cnt);
+        atomicAdd(&smass[cur], mass);
+      } else {
+        hist_flush(hist, cur, cnt, mass);
+      }
+    };
+    for (int c = lane; c <= r; c += 32) {
+      const float v = dev::ex2(row[c] - m) * inv;
+      row[c] = v;
+      const uint32_t bucket = __float_as_uint(v) >> 20;
+      if (bucket != cur) {
+        flush();
+        cur = bucket;
+        cnt = 0;
+        mass = 0.0;
+      }
+      ++cnt;
+      mass += (double)v;
     }
-  };
-  for (int c = lane; c <= r; c += 32) {
-    const float v = dev::ex2(row[c] - m) * inv;
-    row[c] = v;
-    const uint32_t bucket = __float_as_uint(v) >> 20;
-    if (bucket != cur) {
-      flush();
-      cur = bucket;
-      cnt = 0;
-      mass = 0.0;
-    }
-    ++cnt;
-    mass += (double)v;
+    flush();
   }
-  flush();
-  __syncwarp();
-  if (window) {
-    for (int i = lane; i < kWin; i += 32)
-      if (wcount[warp][i]) hist_flush(hist, b_lo + i, wcount[warp][i], wmass[warp][i]);
-  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < kL0Low; i += blockDim.x)
+    if (scount[i]) hist_flush(hist, (uint32_t)i, scount[i], smass[i]);
 }
 
 // Histogram of the entries whose key matches the prefix found so far
 // (level 1: bits 19..8 under the 12-bit prefix; level 2: bits 7..0 under the
-// 24-bit prefix). float4 sweeps over the head's triangle (stride padded to 64).
+// 24-bit prefix). float4 sweeps over the head's triangle (stride padded to
+// 64); each CTA gathers its part in shared memory (dynamic, 16 bytes per
+// bucket) and adds its non-empty buckets to the global histogram.
 __global__ void __launch_bounds__(256) pe_hist_kernel(PeArgs a, int level) {
   const int h = blockIdx.y;
   if (a.route[h] != 1) return;
   const PeState* st = a.state + h;
-  if (st->all) return;
+  if (st->all) return;   // uniform over the CTA
+  extern __shared__ __align__(16) unsigned char hsm[];
+  const int nbk = level == 1 ? kHistL1 : kHistL2;
+  unsigned long long* scount = reinterpret_cast<unsigned long long*>(hsm);
+  double* smass = reinterpret_cast<double*>(hsm + (size_t)nbk * sizeof(unsigned long long));
+  for (int i = threadIdx.x; i < nbk; i += blockDim.x) {
+    scount[i] = 0;
+    smass[i] = 0.0;
+  }
+  __syncthreads();
   const uint32_t prefix = st->prefix;
   const int shift_p = level == 1 ? 20 : 8;
   const int shift_b = level == 1 ? 8 : 0;
   const uint32_t bmask = level == 1 ? 0xFFFu : 0xFFu;
   const float4* tri4 = reinterpret_cast<const float4*>(a.tri_buf + (size_t)h * a.tri_stride);
-  PeHist* hist = a.hist + h;
   const long long n4 = (a.tri + 3) / 4;
   for (long long p = (long long)blockIdx.x * blockDim.x + threadIdx.x; p < n4; p += (long long)gridDim.x * blockDim.x) {
     const float4 v4 = tri4[p];
@@ -269,11 +269,15 @@ __global__ void __launch_bounds__(256) pe_hist_kernel(PeArgs a, int level) {
       const uint32_t key = __float_as_uint(vv[i]);
       if ((key >> shift_p) == prefix) {
         const uint32_t b = (key >> shift_b) & bmask;
-        atomicAdd(&hist->count[b], 1ull);
-        atomicAdd(&hist->mass[b], (double)vv[i]);
+        atomicAdd(&scount[b], 1ull);
+        atomicAdd(&smass[b], (double)vv[i]);
       }
     }
   }
+  __syncthreads();
+  PeHist* hist = a.hist + h;
+  for (int i = threadIdx.x; i < nbk; i += blockDim.x)
+    if (scount[i]) hist_flush(hist, (uint32_t)i, scount[i], smass[i]);
 }
 
 // Walk the buckets of the current level from the largest key down, carrying
@@ -526,10 +530,13 @@ cudaError_t launch_pe(const void* q, const void* k, const Shape& s, char* ws, co
   const int row_ctas = (s.nb + kRowsPerCta - 1) / kRowsPerCta;
   pe_softmax_kernel<<<dim3(row_ctas, s.h_q), 256, 0, st>>>(a);
   pe_find_kernel<<<s.h_q, 1024, 0, st>>>(a, 0);
-  const int hist_ctas = (int)std::min<long long>(1184, (s.tri / 4 + 255) / 256 + 1);
-  pe_hist_kernel<<<dim3(hist_ctas, s.h_q), 256, 0, st>>>(a, 1);
+  const int hist_ctas = (int)std::min<long long>(296, (s.tri / 4 + 255) / 256 + 1);
+  const size_t hsm1 = (size_t)kHistL1 * 16, hsm2 = (size_t)kHistL2 * 16;
+  e = cudaFuncSetAttribute(pe_hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hsm1);
+  if (e != cudaSuccess) return e;
+  pe_hist_kernel<<<dim3(hist_ctas, s.h_q), 256, hsm1, st>>>(a, 1);
   pe_find_kernel<<<s.h_q, 1024, 0, st>>>(a, 1);
-  pe_hist_kernel<<<dim3(hist_ctas, s.h_q), 256, 0, st>>>(a, 2);
+  pe_hist_kernel<<<dim3(hist_ctas, s.h_q), 256, hsm2, st>>>(a, 2);
   pe_find_kernel<<<s.h_q, 1024, 0, st>>>(a, 2);
   pe_tie_count_kernel<<<dim3(row_ctas, s.h_q), 256, 0, st>>>(a);
   pe_tie_scan_kernel<<<s.h_q, 1024, 0, st>>>(a);
