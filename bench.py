@@ -147,17 +147,20 @@ def kernel_source_hash(names):
     return h.hexdigest()[:16]
 
 
-def load_traffic(kernel, src_hash):
-    """DRAM bytes per launch from a committed ncu summary, if it was taken on this source."""
-    p = os.path.join(ROOT, "profiles", "traffic.json")
-    if not os.path.exists(p):
+# dram__bytes_read.sum + dram__bytes_write.sum of one launch, from the ncu
+# capture summarised in profiles/attn_tc_traffic_layerE.md (layer E, default
+# alpha and gamma); reported only for the kernel source it was taken on.
+MEASURED_TRAFFIC = {
+    ("attn_tc_kernel", "E", 1.0, 0.95): {"source_hash": "e58218f1e1abe0d2", "bytes_per_launch": 5.00e12 + 4.34e9},
+}
+
+
+def load_traffic(kernel, src_hash, config, alpha, gamma):
+    """DRAM bytes per launch measured on this kernel source and workload, else None."""
+    e = MEASURED_TRAFFIC.get((kernel, config, float(alpha), float(gamma)))
+    if not e or e["source_hash"] != src_hash:
         return None
-    with open(p) as f:
-        d = json.load(f)
-    e = d.get(kernel)
-    if not e or e.get("source_hash") != src_hash:
-        return None
-    return e.get("bytes_per_launch")
+    return e["bytes_per_launch"]
 
 
 def cpu_cores():
@@ -350,7 +353,7 @@ def run_crisp(args, rank, world, local_rank):
     h2d = int(q_h.numel() * q_h.element_size() + k_h.numel() * k_h.element_size() + v_h.numel() * v_h.element_size())
     d2h = int(out_h.numel() * out_h.element_size())
     src_hash = kernel_source_hash(["attn_tc.cu", "ptx.cuh"])
-    traffic = load_traffic("attn_tc_kernel", src_hash)
+    traffic = load_traffic("attn_tc_kernel", src_hash, args.config, args.alpha, args.gamma)
     # algorithmic HBM bytes of the route pass: K read once, proxy rows of Q,
     # per-(row, tile) partials written and read back, chunk statistics
     nb = cfg.n_blocks
