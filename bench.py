@@ -11,7 +11,9 @@ full-size layer, so no flush is needed between steps. The dense reference and
 the end-to-end number (crisp_prefill through host buffers, copies included)
 are timed the same way. With N > 1 (torchrun) every rank runs its own layer
 (weak scaling, no collective on the data path); the step time is the max over
-ranks and the reported ms/layer divides it by N.
+ranks and the reported ms/layer divides it by N. ``--shard heads`` instead
+splits one layer across the ranks by KV group (strong scaling: each rank draws
+and runs only its groups; the layer's time is the slowest rank's).
 
 ``--impl reference`` times the CPU oracle (float64, host cores) on a bounded
 sample of the same workload and scales it to ms/layer.
@@ -163,6 +165,17 @@ def load_traffic(kernel, src_hash, config, alpha, gamma):
     return e["bytes_per_launch"]
 
 
+def mufu_roofline(exps, ms, clk, sms):
+    """Exponentials per second against the MUFU rate (16 per clock per SM) at the sampled SM clock."""
+    mhz = clk.get("sm_mhz") or clk.get("sm_max_mhz")
+    if not mhz or ms <= 0:
+        return None
+    peak = 16.0 * sms * mhz * 1e6
+    achieved = exps / (ms * 1e-3)
+    return {"exps": int(exps), "achieved_per_s": round(achieved / 1e12, 3), "peak_per_s": round(peak / 1e12, 3),
+            "unit": "T exp2/s", "frac": round(achieved / peak, 4), "clock_mhz": mhz}
+
+
 def cpu_cores():
     try:
         from threadpoolctl import threadpool_info
@@ -233,18 +246,34 @@ def run_crisp(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
     import long_context_prefill_last_b200 as crisp
+    from long_context_prefill_last_b200 import shard
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     c = S.CONFIGS[args.config]
-    layer = S.generate(c, threads=min(32, os.cpu_count() or 8))
-    q_h, k_h, v_h = S.to_torch(layer)
+    threads = min(32, os.cpu_count() or 8)
+    heads_mode = args.shard == "heads" and world > 1
+    if heads_mode:
+        # one layer split by KV group: this rank draws and runs only its groups
+        if world > c.h_kv:
+            raise SystemExit(f"--shard heads needs at most {c.h_kv} ranks for layer {args.config}")
+        g_lo, g_hi = shard.kv_group_range(c.h_kv, world, rank)
+        arrays = S.generate_slice(c, g_lo, g_hi, threads=threads)
+        h_q, h_kv = (g_hi - g_lo) * c.group, g_hi - g_lo
+        if c.dtype == "bf16":
+            q_h, k_h, v_h = (torch.from_numpy(a).view(torch.bfloat16) for a in arrays)
+        else:
+            q_h, k_h, v_h = (torch.from_numpy(a) for a in arrays)
+    else:
+        layer = S.generate(c, threads=threads)
+        q_h, k_h, v_h = S.to_torch(layer)
+        h_q, h_kv = c.h_q, c.h_kv
     q_h, k_h, v_h = q_h.pin_memory(), k_h.pin_memory(), v_h.pin_memory()
     q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
     out = torch.empty_like(q)
     out_h = torch.empty(q.shape, dtype=q.dtype).pin_memory()
     dtype = crisp.FP32 if c.dtype == "fp32" else crisp.BF16
-    cfg = crisp.Config(n=c.n, h_q=c.h_q, h_kv=c.h_kv, d=c.d, dtype=dtype, alpha=args.alpha, gamma=args.gamma)
+    cfg = crisp.Config(n=c.n, h_q=h_q, h_kv=h_kv, d=c.d, dtype=dtype, alpha=args.alpha, gamma=args.gamma)
     cfg.allocate_workspace(dev)
     ix = crisp.IndexBuffers(cfg, dev)
     stream = torch.cuda.current_stream(dev)
@@ -266,7 +295,7 @@ def run_crisp(args, rank, world, local_rank):
     route = ix.route.cpu().numpy()
     tiles = kept_tiles(route, ix.vs_mask.cpu().numpy().view(np.uint32), ix.pe_mask.cpu().numpy().view(np.uint32),
                        cfg.n_blocks)
-    causal_tiles = c.h_q * cfg.n_blocks * (cfg.n_blocks + 1) // 2
+    causal_tiles = h_q * cfg.n_blocks * (cfg.n_blocks + 1) // 2
 
     clocks = ClockSampler(local_rank)
     clocks.start()
@@ -287,8 +316,8 @@ def run_crisp(args, rank, world, local_rank):
     crisp.raise_on_device_status(cfg, stream, "timed steps")
 
     # --- timed: the route pass alone (proxy map + finalisation + route/VS masses)
-    r_out = torch.empty(c.h_q, dtype=torch.int32, device=dev)
-    c_out = torch.empty(c.h_q, dtype=torch.float32, device=dev)
+    r_out = torch.empty(h_q, dtype=torch.int32, device=dev)
+    c_out = torch.empty(h_q, dtype=torch.float32, device=dev)
     crisp.route(q, k, cfg, r_out, c_out, stream)
     torch.cuda.synchronize(dev)
     rev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
@@ -335,49 +364,69 @@ def run_crisp(args, rank, world, local_rank):
     crisp.raise_on_device_status(cfg, stream, "e2e")
     clk = clocks.stop()
 
-    # max over ranks
-    vals = torch.tensor([statistics.mean(step_ms), statistics.mean(att_ms), statistics.mean(sel_ms),
-                         statistics.mean(dense_ms), statistics.mean(e2e_ms), statistics.mean(route_ms)],
-                        dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-    step_m, att_m, sel_m, dense_m, e2e_m, route_m = vals.tolist()
-    if rank != 0:
-        return None
-
+    # per-rank work of this rank's launches
     peaks, peak_src = load_peaks()
     tflops_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    hbm_peak = peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"])
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    att_l, sel_l, route_l = statistics.mean(att_ms), statistics.mean(sel_ms), statistics.mean(route_ms)
     flops = 4.0 * c.d * 128 * 128 * tiles          # computed-tile work of one attention launch
-    achieved = flops / (att_m * 1e-3) / 1e12
-    dense_flops = 4.0 * c.d * 128 * 128 * causal_tiles
-    h2d = int(q_h.numel() * q_h.element_size() + k_h.numel() * k_h.element_size() + v_h.numel() * v_h.element_size())
-    d2h = int(out_h.numel() * out_h.element_size())
-    src_hash = kernel_source_hash(["attn_tc.cu", "ptx.cuh"])
-    traffic = load_traffic("attn_tc_kernel", src_hash, args.config, args.alpha, args.gamma)
     # algorithmic HBM bytes of the route pass: K read once, proxy rows of Q,
     # per-(row, tile) partials written and read back, chunk statistics
     nb = cfg.n_blocks
-    rows = c.h_q * 64
-    route_bytes = (c.h_kv * c.n * c.d * 2 + rows * c.d * 2 + 2 * rows * nb * 8
+    rows = h_q * 64
+    route_bytes = (h_kv * c.n * c.d * 2 + rows * c.d * 2 + 2 * rows * nb * 8
                    + rows * ((nb + 7) // 8) * 24)
     # selection (PE heads): their Q and their groups' K pooled once, the pooled
     # map written once and swept by the softmax (read+write), two histogram
     # passes and the mask pass (reads), plus the PE masks written
     n_pe = int((route == 1).sum())
-    g_pe = len({h // c.group for h in range(c.h_q) if route[h] == 1})
+    g_pe = len({h // c.group for h in range(h_q) if route[h] == 1})
     tri = nb * (nb + 1) // 2
     pe_bytes = (n_pe + g_pe) * c.n * c.d * 2 + n_pe * tri * 4 * 6 + n_pe * nb * cfg.words * 4
-    hbm_peak = peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"])
+    pe_ms = max(sel_l - route_l, 1e-6)
+    mufu = mufu_roofline(h_q * cfg.last_q * c.n, route_l, clk, sms)
+
+    # across ranks: times are the maximum; rates the minimum (slowest rank);
+    # with the layer split by KV group, tile and head counts add up
+    vals = torch.tensor([statistics.mean(step_ms), att_l, sel_l, statistics.mean(dense_ms),
+                         statistics.mean(e2e_ms), route_l], dtype=torch.float64, device=dev)
+    rates = torch.tensor([flops / (att_l * 1e-3) / 1e12, route_bytes / (route_l * 1e-3) / 1e9,
+                          pe_bytes / (pe_ms * 1e-3) / 1e9, (mufu or {}).get("frac", 0.0)],
+                         dtype=torch.float64, device=dev)
+    counts = torch.tensor([tiles, causal_tiles, int((route == 0).sum()), int((route == 1).sum())],
+                          dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+        dist.all_reduce(rates, op=dist.ReduceOp.MIN)
+        if heads_mode:
+            dist.all_reduce(counts, op=dist.ReduceOp.SUM)
+    step_m, att_m, sel_m, dense_m, e2e_m, route_m = vals.tolist()
+    achieved, route_gbs, pe_gbs, mufu_frac = rates.tolist()
+    tiles_all, causal_all, heads_vs, heads_pe = (int(x) for x in counts.tolist())
+    if rank != 0:
+        return None
+    if mufu is not None:
+        mufu["frac"] = round(mufu_frac, 4)
+    dense_flops = 4.0 * c.d * 128 * 128 * causal_tiles
+    h2d = int(q_h.numel() * q_h.element_size() + k_h.numel() * k_h.element_size() + v_h.numel() * v_h.element_size())
+    d2h = int(out_h.numel() * out_h.element_size())
+    src_hash = kernel_source_hash(["attn_tc.cu", "ptx.cuh"])
+    traffic = (load_traffic("attn_tc_kernel", src_hash, args.config, args.alpha, args.gamma)
+               if not heads_mode else None)
+    # whole-job ms per layer: independent layers per GPU divide by the GPUs;
+    # one layer split by KV group takes the slowest rank's time
+    per_layer = 1 if heads_mode else world
     res = {
         "metric": METRIC,
-        "value": round(step_m / world, 4),
+        "value": round(step_m / per_layer, 4),
         "unit": "ms/layer",
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
         "ms_per_step": round(step_m, 4),
         "higher_is_better": False,
-        "scaling": "weak",
+        "scaling": "strong" if heads_mode else "weak",
         "vs_baseline": None,
         "dtype": "bf16" if c.dtype == "bf16" else "f32",
         "data": ("synthetic (seeded Gaussian heads with planted sink/vertical/slash structure"
@@ -385,13 +434,15 @@ def run_crisp(args, rank, world, local_rank):
                  + "; no datasets or weights)"),
         "config": {"workload": f"layer {args.config}: {c.desc}", "h_q": c.h_q, "h_kv": c.h_kv, "seq_len": c.n,
                    "alpha": args.alpha, "gamma": args.gamma,
-                   "head_dim": c.d, "batch": 1, "parallelism": f"independent layer per GPU x{world}",
+                   "head_dim": c.d, "batch": 1,
+                   "parallelism": (f"one layer split by KV group over {world} GPUs (no exchange)" if heads_mode
+                                   else f"independent layer per GPU x{world}"),
                    "l2": "inputs (>= 6 GiB at 512K) far exceed the 126 MB L2; no flush between steps"},
         "speedup_vs_dense": round(dense_m / step_m, 4),
         "dense_ms_per_layer": round(dense_m, 4),
         "stages_ms": {"proxy_route_select": round(sel_m, 4), "sparse_attention": round(att_m, 4)},
-        "density": {"computed_tiles": tiles, "causal_tiles": causal_tiles, "fraction": round(tiles / causal_tiles, 4),
-                    "heads_vs": int((route == 0).sum()), "heads_pe": int((route == 1).sum())},
+        "density": {"computed_tiles": tiles_all, "causal_tiles": causal_all,
+                    "fraction": round(tiles_all / causal_all, 4), "heads_vs": heads_vs, "heads_pe": heads_pe},
         "pages_speedup_context": f"{PAGES_SPEEDUP_512K}x at 512K tokens on one H100 (pages' figure, not comparable)",
         "roofline": {"kernel": "attn_tc_kernel (block-sparse attention)", "bound": "tensor",
                      "achieved": round(achieved, 2), "peak": tflops_peak, "unit": "TFLOP/s",
@@ -401,15 +452,18 @@ def run_crisp(args, rank, world, local_rank):
         "dense_tflops": round(dense_flops / (dense_m * 1e-3) / 1e12, 2),
         "route_roofline": {"stage": "crisp_route (proxy_tc_kernel + finalize + VS masses)", "bound": "hbm",
                            "ms": round(route_m, 4), "algorithmic_bytes": route_bytes,
-                           "achieved": round(route_bytes / (route_m * 1e-3) / 1e9, 1), "peak": hbm_peak,
-                           "unit": "GB/s", "frac": round(route_bytes / (route_m * 1e-3) / 1e9 / hbm_peak, 4)},
+                           "achieved": round(route_gbs, 1), "peak": hbm_peak,
+                           "unit": "GB/s", "frac": round(route_gbs / hbm_peak, 4),
+                           # the proxy's exponentials (h_q x 64 x n) against MUFU at 16 per clock per SM
+                           # and the median SM clock sampled under load
+                           "mufu": mufu},
         "selection_roofline": {"stage": "PE pooling, pooled map, gamma cut, masks (select minus route)",
                                "bound": "hbm", "ms": round(max(sel_m - route_m, 1e-6), 4),
                                "algorithmic_bytes": pe_bytes,
-                               "achieved": round(pe_bytes / (max(sel_m - route_m, 1e-6) * 1e-3) / 1e9, 1),
+                               "achieved": round(pe_gbs, 1),
                                "peak": hbm_peak, "unit": "GB/s",
-                               "frac": round(pe_bytes / (max(sel_m - route_m, 1e-6) * 1e-3) / 1e9 / hbm_peak, 4)},
-        "e2e": {"value": round(e2e_m / world, 4), "unit": "ms/layer", "h2d_bytes_per_step": h2d,
+                               "frac": round(pe_gbs / hbm_peak, 4)},
+        "e2e": {"value": round(e2e_m / per_layer, 4), "unit": "ms/layer", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "api": "crisp_prefill with pinned host buffers"},
         "gpu_launches": KERNELS_PER_STEP * args.steps,
         "clocks": clk,
@@ -464,6 +518,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--alpha", type=float, default=1.0, help="Eq. (4) noise-floor multiplier")
     ap.add_argument("--gamma", type=float, default=0.95, help="PE cumulative coverage")
+    ap.add_argument("--shard", choices=["layers", "heads"], default="layers",
+                    help="with N > 1 GPUs: an independent layer per GPU (weak scaling, default) or one layer "
+                         "split by KV group (strong scaling)")
     ap.add_argument("--only", choices=["select", "attend", "dense", "prefill", "route"],
                     help="profiling mode: time one stage alone (no contract line)")
     ap.add_argument("--n", type=int, help="profiling mode: scaled sequence length")

@@ -367,6 +367,38 @@ def generate(cfg: LayerConfig, threads: int = 8, with_v: bool = True) -> Layer:
     return Layer(cfg, q, k, v, st)
 
 
+def generate_slice(cfg: LayerConfig, g_lo: int, g_hi: int, threads: int = 8, with_v: bool = True):
+    """KV groups [g_lo, g_hi) of the layer and their query heads, exactly as
+    the same rows of ``generate(cfg)``: (q [(g_hi-g_lo)*G, n, d], k, v
+    [g_hi-g_lo, n, d]) in the layer's storage type. Every tensor is drawn from
+    its own seed, so a rank can draw only its shard."""
+    if not 0 <= g_lo < g_hi <= cfg.h_kv:
+        raise ValueError("bad group range")
+    n, d, G = cfg.n, cfg.d, cfg.group
+    bf16 = cfg.dtype == "bf16"
+    st = {g: group_structure(cfg, g) for g in cfg.planted_groups if g_lo <= g < g_hi}
+    dt = np.uint16 if bf16 else np.float32
+    ng = g_hi - g_lo
+    q = np.empty((ng * G, n, d), dtype=dt)
+    k = np.empty((ng, n, d), dtype=dt)
+    v = np.empty((ng, n, d), dtype=dt) if with_v else np.zeros((ng, 0, d), dtype=dt)
+
+    def store(dst, i, x):
+        dst[i] = f32_to_bf16_bits(x) if bf16 else x
+
+    jobs = []
+    for g in range(g_lo, g_hi):
+        jobs.append(lambda g=g: store(k, g - g_lo, _gen_k(cfg, g, st.get(g))))
+        if with_v:
+            jobs.append(lambda g=g: store(v, g - g_lo, _gen_v(cfg, g)))
+        for h in range(g * G, (g + 1) * G):
+            jobs.append(lambda h=h, g=g: store(q, h - g_lo * G, _gen_q(cfg, h, st.get(g))))
+    with ThreadPoolExecutor(max_workers=max(1, threads)) as ex:
+        for f in [ex.submit(j) for j in jobs]:
+            f.result()
+    return q, k, v
+
+
 def to_torch(layer: Layer):
     """(q, k, v) as CPU torch tensors of the layer's dtype (views, no copy)."""
     import torch

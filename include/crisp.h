@@ -137,6 +137,34 @@ crisp_status crisp_attend(const void* q, const void* k, const void* v, void* out
 crisp_status crisp_prefill(const void* q, const void* k, const void* v, void* out,
                            const crisp_cfg* cfg, void* stream);
 
+/* Algorithm 1 for `batch` independent sequences of one length (no
+ * counterpart in the paper, which treats one prompt at a time). q and out
+ * are [batch][h_q][n][d], k and v [batch][h_kv][n][d], contiguous; cfg
+ * describes ONE sequence. Every stage works per head and the sequences are
+ * laid out head after head, so the call is crisp_prefill on the folded shape
+ * (batch*h_q query heads, batch*h_kv key/value heads; query head b*h_q + j
+ * reads key/value head b*h_kv + j / (h_q/h_kv), i.e. its own sequence's).
+ * cfg->workspace must hold crisp_workspace_size_batch(cfg, batch) bytes.
+ * batch < 1: CRISP_ERR_INVALID_ARG; a folded shape outside the limits of a
+ * single call (h_q * batch <= 1024): CRISP_ERR_SHAPE. */
+crisp_status crisp_prefill_batch(const void* q, const void* k, const void* v, void* out,
+                                 const crisp_cfg* cfg, int32_t batch, void* stream);
+
+/* Workspace bytes crisp_prefill_batch needs for `batch` sequences of cfg's shape. */
+crisp_status crisp_workspace_size_batch(const crisp_cfg* cfg, int32_t batch, size_t* bytes);
+
+/* Algorithm 1 for `count` sequences of different lengths (no counterpart in
+ * the paper). Sequence i has its own tensors q[i], out[i] ([h_q][n[i]][d])
+ * and k[i], v[i] ([h_kv][n[i]][d]); q, k, v, out and n are HOST arrays of
+ * `count` entries (device pointers inside q..out). Each length obeys the
+ * rules of cfg->n; cfg->n itself is ignored. The sequences run one after
+ * another on `stream` and share cfg's workspace, which must hold
+ * crisp_workspace_size for the longest one. Arguments are checked for every
+ * sequence before anything is launched; on an error nothing runs. */
+crisp_status crisp_prefill_varlen(const void* const* q, const void* const* k, const void* const* v,
+                                  void* const* out, const int32_t* n, int32_t count,
+                                  const crisp_cfg* cfg, void* stream);
+
 /* Exact dense causal attention with the same kernels (the speed reference). */
 crisp_status crisp_dense_attention(const void* q, const void* k, const void* v, void* out,
                                    const crisp_cfg* cfg, void* stream);

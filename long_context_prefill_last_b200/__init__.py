@@ -33,7 +33,8 @@ STATUS_NAMES = {
 # every function include/crisp.h declares
 SYMBOLS = ["crisp_cfg_init", "crisp_workspace_size", "crisp_index_dims", "crisp_route", "crisp_select",
            "crisp_attend", "crisp_prefill", "crisp_dense_attention", "crisp_device_status",
-           "crisp_status_string", "crisp_version", "crisp_route_noalloc", "crisp_exp2_selftest"]
+           "crisp_status_string", "crisp_version", "crisp_route_noalloc", "crisp_exp2_selftest",
+           "crisp_prefill_batch", "crisp_workspace_size_batch", "crisp_prefill_varlen"]
 
 
 def library_path() -> str:
@@ -87,6 +88,11 @@ def lib() -> ctypes.CDLL:
         L.crisp_select.argtypes = [vp, vp, cfgp, ctypes.POINTER(_Index), vp]
         L.crisp_attend.argtypes = [vp, vp, vp, vp, cfgp, ctypes.POINTER(_Index), vp]
         L.crisp_prefill.argtypes = [vp, vp, vp, vp, cfgp, vp]
+        L.crisp_prefill_batch.argtypes = [vp, vp, vp, vp, cfgp, ctypes.c_int32, vp]
+        L.crisp_workspace_size_batch.argtypes = [cfgp, ctypes.c_int32, ctypes.POINTER(ctypes.c_size_t)]
+        L.crisp_prefill_varlen.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.POINTER(vp),
+                                           ctypes.POINTER(vp), ctypes.POINTER(ctypes.c_int32), ctypes.c_int32,
+                                           cfgp, vp]
         L.crisp_dense_attention.argtypes = [vp, vp, vp, vp, cfgp, vp]
         L.crisp_device_status.argtypes = [cfgp, vp, ctypes.POINTER(ctypes.c_int32)]
         L.crisp_status_string.argtypes = [ctypes.c_int]
@@ -147,15 +153,26 @@ class Config:
             c.workspace_bytes = self.workspace.numel() * self.workspace.element_size()
         return c
 
-    def allocate_workspace(self, device="cuda"):
+    def allocate_workspace(self, device="cuda", batch: int = 1, max_n: Optional[int] = None):
+        """Device workspace for this shape; `batch` sequences (crisp_prefill_batch)
+        or sequences up to `max_n` tokens (crisp_prefill_varlen)."""
         import torch
-        self.workspace = torch.empty(workspace_size(self), dtype=torch.uint8, device=device)
+        c = dataclasses.replace(self, n=max_n) if max_n is not None else self
+        nbytes = workspace_size(c) if batch == 1 else workspace_size_batch(c, batch)
+        self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=device)
         return self.workspace
 
 
 def workspace_size(cfg: Config) -> int:
     out = ctypes.c_size_t(0)
     _check(lib().crisp_workspace_size(ctypes.byref(cfg._c()), ctypes.byref(out)), "crisp_workspace_size")
+    return out.value
+
+
+def workspace_size_batch(cfg: Config, batch: int) -> int:
+    out = ctypes.c_size_t(0)
+    _check(lib().crisp_workspace_size_batch(ctypes.byref(cfg._c()), int(batch), ctypes.byref(out)),
+           "crisp_workspace_size_batch")
     return out.value
 
 
@@ -231,6 +248,24 @@ def attend(q, k, v, out, cfg: Config, index: IndexBuffers, stream=None) -> None:
 def prefill(q, k, v, out, cfg: Config, stream=None) -> None:
     _check(lib().crisp_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(out), ctypes.byref(cfg._c()), _stream(stream)),
            "crisp_prefill")
+
+
+def prefill_batch(q, k, v, out, cfg: Config, stream=None) -> None:
+    """crisp_prefill_batch: q/out [batch, h_q, n, d], k/v [batch, h_kv, n, d]; cfg is one sequence's."""
+    _check(lib().crisp_prefill_batch(_ptr(q), _ptr(k), _ptr(v), _ptr(out), ctypes.byref(cfg._c()), int(q.shape[0]),
+                                     _stream(stream)), "crisp_prefill_batch")
+
+
+def prefill_varlen(qs, ks, vs, outs, cfg: Config, stream=None) -> None:
+    """crisp_prefill_varlen: per-sequence tensors qs[i] [h_q, n_i, d], ks/vs[i] [h_kv, n_i, d]."""
+    cnt = len(qs)
+    if not (len(ks) == len(vs) == len(outs) == cnt):
+        raise ValueError("q, k, v and out lists differ in length")
+    arr = ctypes.c_void_p * cnt
+    n = (ctypes.c_int32 * cnt)(*[int(t.shape[1]) for t in qs])
+    _check(lib().crisp_prefill_varlen(arr(*[_ptr(t) for t in qs]), arr(*[_ptr(t) for t in ks]),
+                                      arr(*[_ptr(t) for t in vs]), arr(*[_ptr(t) for t in outs]), n, cnt,
+                                      ctypes.byref(cfg._c()), _stream(stream)), "crisp_prefill_varlen")
 
 
 def dense_attention(q, k, v, out, cfg: Config, stream=None) -> None:

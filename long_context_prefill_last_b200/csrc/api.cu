@@ -213,6 +213,32 @@ static crisp_status prepare(const crisp_cfg* cfg, const void* q, const void* k, 
   return check_ws(cfg, *L);
 }
 
+// Algorithm 1 on one layer; `clear` resets the device status word first.
+static crisp_status prefill_impl(const void* q, const void* k, const void* v, void* out, const crisp_cfg* cfg,
+                                 cudaStream_t st, bool clear) {
+  Shape s;
+  WsLayout L;
+  crisp_status r = prepare(cfg, q, k, v, out, true, &s, &L);
+  if (r != CRISP_OK) return r;
+  char* ws = static_cast<char*>(cfg->workspace);
+  if (clear) CRISP_TRY(cudaMemsetAsync(ws + L.status, 0, 32, st));
+  IndexPtrs ix = internal_index(ws, L);
+  r = run_index(q, k, s, ws, L, ix, true, st);
+  if (r != CRISP_OK) return r;
+  return run_attention(q, k, v, out, s, ws, L, ix.route, ix.vs_mask, ix.pe_mask, false, st);
+}
+
+// One sequence's cfg -> the cfg of `batch` sequences laid out head after head.
+static crisp_status fold_batch(const crisp_cfg* cfg, int32_t batch, crisp_cfg* folded) {
+  if (cfg == nullptr || batch < 1) return CRISP_ERR_INVALID_ARG;
+  const long long hq = (long long)cfg->h_q * batch, hkv = (long long)cfg->h_kv * batch;
+  if (hq > INT32_MAX || hkv > INT32_MAX) return CRISP_ERR_INVALID_ARG;
+  *folded = *cfg;
+  folded->h_q = (int32_t)hq;
+  folded->h_kv = (int32_t)hkv;
+  return CRISP_OK;
+}
+
 }  // namespace crisp
 
 using namespace crisp;
@@ -304,17 +330,48 @@ crisp_status crisp_attend(const void* q, const void* k, const void* v, void* out
 
 crisp_status crisp_prefill(const void* q, const void* k, const void* v, void* out, const crisp_cfg* cfg,
                            void* stream) {
-  Shape s;
-  WsLayout L;
-  crisp_status r = prepare(cfg, q, k, v, out, true, &s, &L);
+  return prefill_impl(q, k, v, out, cfg, static_cast<cudaStream_t>(stream), true);
+}
+
+crisp_status crisp_workspace_size_batch(const crisp_cfg* cfg, int32_t batch, size_t* bytes) {
+  crisp_cfg f;
+  crisp_status r = fold_batch(cfg, batch, &f);
   if (r != CRISP_OK) return r;
+  return crisp_workspace_size(&f, bytes);
+}
+
+crisp_status crisp_prefill_batch(const void* q, const void* k, const void* v, void* out, const crisp_cfg* cfg,
+                                 int32_t batch, void* stream) {
+  crisp_cfg f;
+  crisp_status r = fold_batch(cfg, batch, &f);
+  if (r != CRISP_OK) return r;
+  return prefill_impl(q, k, v, out, &f, static_cast<cudaStream_t>(stream), true);
+}
+
+crisp_status crisp_prefill_varlen(const void* const* q, const void* const* k, const void* const* v,
+                                  void* const* out, const int32_t* n, int32_t count, const crisp_cfg* cfg,
+                                  void* stream) {
+  if (cfg == nullptr || q == nullptr || k == nullptr || v == nullptr || out == nullptr || n == nullptr || count < 1)
+    return CRISP_ERR_INVALID_ARG;
+  // every sequence is checked before anything is launched
+  for (int32_t i = 0; i < count; ++i) {
+    crisp_cfg c = *cfg;
+    c.n = n[i];
+    Shape s;
+    WsLayout L;
+    crisp_status r = prepare(&c, q[i], k[i], v[i], out[i], true, &s, &L);
+    if (r != CRISP_OK) return r;
+  }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  char* ws = static_cast<char*>(cfg->workspace);
-  CRISP_TRY(cudaMemsetAsync(ws + L.status, 0, 32, st));
-  IndexPtrs ix = internal_index(ws, L);
-  r = run_index(q, k, s, ws, L, ix, true, st);
-  if (r != CRISP_OK) return r;
-  return run_attention(q, k, v, out, s, ws, L, ix.route, ix.vs_mask, ix.pe_mask, false, st);
+  for (int32_t i = 0; i < count; ++i) {
+    crisp_cfg c = *cfg;
+    c.n = n[i];
+    // the status word is cleared by the first sequence only, so a device-side
+    // failure of any sequence stays visible (later kernels see it and stop)
+    crisp_status r = prefill_impl(q[i], k[i], v[i], out[i], &c, st, i == 0);
+    if (r != CRISP_OK) return r;
+  }
+  return CRISP_OK;
 }
 
 crisp_status crisp_dense_attention(const void* q, const void* k, const void* v, void* out, const crisp_cfg* cfg,

@@ -149,3 +149,38 @@ def test_status_strings():
     assert crisp.status_string(0) == "ok"
     assert "timed out" in crisp.status_string(9)
     assert crisp.lib().crisp_version() >= 100
+
+
+def test_batch_and_varlen_validation_before_any_launch():
+    L = crisp.lib()
+    one = crisp.Config(n=4096, h_q=8, h_kv=2)
+    # a batch of b sequences needs the workspace of the folded shape
+    for b in (1, 2, 3):
+        folded = crisp.Config(n=4096, h_q=8 * b, h_kv=2 * b)
+        assert crisp.workspace_size_batch(one, b) == crisp.workspace_size(folded)
+    out = ctypes.c_size_t(0)
+    assert L.crisp_workspace_size_batch(ctypes.byref(one._c()), 0, ctypes.byref(out)) == 1
+    assert L.crisp_prefill_batch(0x10000, 0x20000, 0x30000, 0x40000, ctypes.byref(one._c()), 0, None) == 1
+    # the folded shape obeys the single-call limits (h_q <= 1024)
+    assert L.crisp_prefill_batch(0x10000, 0x20000, 0x30000, 0x40000, ctypes.byref(one._c()), 129, None) == 2
+    # without a workspace: rejected before anything runs
+    assert L.crisp_prefill_batch(0x10000, 0x20000, 0x30000, 0x40000, ctypes.byref(one._c()), 2, None) == 5
+
+    vp = ctypes.c_void_p
+    arr = vp * 2
+    q, k, v, o = arr(0x10000, 0x50000), arr(0x20000, 0x60000), arr(0x30000, 0x70000), arr(0x40000, 0x80000)
+    cfg = crisp.Config(n=4096, h_q=8, h_kv=2)
+    cfg.workspace = _FakeTensor(0x100000, 1 << 40)
+    c = cfg._c()
+    n_ok = (ctypes.c_int32 * 2)(4096, 2048)
+    n_bad = (ctypes.c_int32 * 2)(4096, 1000)       # not a multiple of 128
+    fn = L.crisp_prefill_varlen
+    assert fn(q, k, v, o, n_ok, 0, ctypes.byref(c), None) == 1            # no sequences
+    assert fn(None, k, v, o, n_ok, 2, ctypes.byref(c), None) == 1         # missing array
+    assert fn(q, k, v, o, None, 2, ctypes.byref(c), None) == 1            # missing lengths
+    assert fn(q, k, v, o, n_bad, 2, ctypes.byref(c), None) == 2           # second length invalid: nothing runs
+    q_bad = arr(0x10000, 0x50008)                                         # second q misaligned
+    assert fn(q_bad, k, v, o, n_ok, 2, ctypes.byref(c), None) == 4
+    small = crisp.Config(n=2048, h_q=8, h_kv=2)
+    small.workspace = _FakeTensor(0x100000, crisp.workspace_size(small))  # too small for n=4096
+    assert fn(q, k, v, o, n_ok, 2, ctypes.byref(small._c()), None) == 5

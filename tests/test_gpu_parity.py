@@ -277,6 +277,35 @@ def test_repeat_calls_are_deterministic():
     assert torch.equal(o1, o2)
 
 
+def test_batch_and_varlen_match_single_calls():
+    # two sequences of one length as a batch, and three lengths as varlen: each
+    # output equals the single-sequence call (every stage works per head)
+    la = S.generate(S.scaled("B", n=2048, h_q=8, h_kv=2))
+    lb = S.generate(S.scaled("C_cliff", n=2048, h_q=8, h_kv=2))
+    lc = S.generate(S.scaled("B", n=1024, h_q=8, h_kv=2, config_id=977))
+    (qa, ka, va), (qb, kb, vb), (qc, kc, vc) = device_layer(la), device_layer(lb), device_layer(lc)
+    singles = []
+    for (q, k, v), lay in (((qa, ka, va), la), ((qb, kb, vb), lb), ((qc, kc, vc), lc)):
+        cfg = make_cfg(lay)
+        o = torch.empty_like(q)
+        crisp.prefill(q, k, v, o, cfg)
+        crisp.raise_on_device_status(cfg)
+        singles.append(o)
+    cfgb = crisp.Config(n=2048, h_q=8, h_kv=2)
+    cfgb.allocate_workspace(batch=2)
+    q, k, v = torch.stack([qa, qb]), torch.stack([ka, kb]), torch.stack([va, vb])
+    out = torch.empty_like(q)
+    crisp.prefill_batch(q, k, v, out, cfgb)
+    crisp.raise_on_device_status(cfgb, where="prefill_batch")
+    assert torch.equal(out[0], singles[0]) and torch.equal(out[1], singles[1])
+    cfgv = crisp.Config(n=2048, h_q=8, h_kv=2)
+    cfgv.allocate_workspace(max_n=2048)
+    outs = [torch.empty_like(qc), torch.empty_like(qa), torch.empty_like(qb)]
+    crisp.prefill_varlen([qc, qa, qb], [kc, ka, kb], [vc, va, vb], outs, cfgv)
+    crisp.raise_on_device_status(cfgv, where="prefill_varlen")
+    assert torch.equal(outs[0], singles[2]) and torch.equal(outs[1], singles[0]) and torch.equal(outs[2], singles[1])
+
+
 # ----------------------------------------------------------------------------- full-size layers
 
 @pytest.mark.parametrize("name", ["B", "C", "D", "E", "E_cliff"])

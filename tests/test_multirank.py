@@ -59,3 +59,48 @@ def test_two_rank_gloo_max_and_partition():
     for rank, t, obj in res:
         assert t == 11.0
         assert obj == [(0, 16), (16, 32)]
+
+
+def _slice_worker(rank, world, port, q):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    import crisp_synth as S
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        # each rank draws only its KV groups of one layer (the --shard heads
+        # path of bench.py); gathered, the shards are the whole layer
+        cfg = S.scaled("C_cliff", n=1024, h_q=8, h_kv=4)
+        lo, hi = shard.kv_group_range(cfg.h_kv, world, rank)
+        qs, ks, _ = S.generate_slice(cfg, lo, hi, threads=2, with_v=False)
+        gq = [None] * world
+        gk = [None] * world
+        dist.all_gather_object(gq, qs)
+        dist.all_gather_object(gk, ks)
+        # timings aggregate as the slowest rank, counts add up
+        t = torch.tensor([5.0 + rank], dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        cnt = torch.tensor([float(hi - lo)], dtype=torch.float64)
+        dist.all_reduce(cnt, op=dist.ReduceOp.SUM)
+        if rank == 0:
+            full = S.generate(cfg, with_v=False)
+            ok = bool((np.concatenate(gq) == full.q).all() and (np.concatenate(gk) == full.k).all())
+            q.put((ok, float(t.item()), float(cnt.item())))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_rank_gloo_head_shards_rebuild_the_layer():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_slice_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    ok, t, cnt = q.get(timeout=180)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert ok and t == 6.0 and cnt == 4.0

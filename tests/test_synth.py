@@ -89,3 +89,14 @@ def test_cliff_sink_fraction_formula():
     w_sink = math.exp(dl)
     rest = (n - 1) * math.exp(0.5) * math.exp(sig * sig / 2)
     assert abs(w_sink / (w_sink + rest) - f) < 1e-12
+
+
+def test_generate_slice_matches_the_full_layer():
+    for base in ("B", "C_cliff"):
+        cfg = S.scaled(base, n=1024, h_q=8, h_kv=4)
+        full = S.generate(cfg)
+        G = cfg.group
+        for lo, hi in ((0, 1), (1, 3), (2, 4)):
+            q, k, v = S.generate_slice(cfg, lo, hi, threads=2)
+            assert (q == full.q[lo * G:hi * G]).all()
+            assert (k == full.k[lo:hi]).all() and (v == full.v[lo:hi]).all()
