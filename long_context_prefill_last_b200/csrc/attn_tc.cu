@@ -8,7 +8,10 @@
 //
 // One CTA per (pair of adjacent 128-row query tiles A = I, B = I-1, query
 // head); the K/V tiles of the union of their schedules stream once through
-// shared memory and serve both. 12 warps in three warpgroups:
+// shared memory and serve both. The grid runs KV group by KV group (heaviest
+// pairs first within a group): the CTAs resident at any time then read one
+// or two KV heads' keys and values, which stay in L2 between them (at
+// 512K tokens this cut DRAM reads from 5.0 TB to 1.9 TB per launch). 12 warps in three warpgroups:
 //   warp 0       TMA producer: Q_A, Q_B once, then K (3-stage ring) and V (2-stage ring)
 //   warp 1       TMEM allocation; one thread issues every tcgen05.mma
 //   warps 2, 3   idle (they complete the first warpgroup)
@@ -136,8 +139,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   uint32_t* tmem_ptr_smem = reinterpret_cast<uint32_t*>(sgen + OFF_TMEMPTR);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int h = blockIdx.x % a.h_q;
-  const int pair = blockIdx.x / a.h_q;                   // heaviest pairs first
+  // KV group by KV group (CTAs that run together share K/V through L2),
+  // heaviest pairs first within a group, the group's query heads adjacent
+  const int per_group = a.n_pairs * a.group;
+  const int g_major = blockIdx.x / per_group;
+  const int rem = blockIdx.x - g_major * per_group;
+  const int pair = rem / a.group;
+  const int h = g_major * a.group + rem % a.group;
   Sched sc;
   sc.IA = (a.nb - 1) - 2 * pair;
   sc.IB = sc.IA - 1;
