@@ -33,6 +33,7 @@ WsLayout ws_layout(const Shape& s) {
   L.qbar = take(hq * nb * kHeadDim * 4);
   L.kbar = take(hkv * nb * kHeadDim * 4);
   L.tri = take(hq * (size_t)s.tri_stride * 4);
+  L.tri_stats = take(hq * nb * (size_t)((s.nb + 63) / 64) * 16);
   L.hist = take(hq * sizeof(PeHist));
   L.pe_state = take(hq * sizeof(PeState));
   L.tie_rows = take(hq * nb * 4);

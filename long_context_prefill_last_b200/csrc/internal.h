@@ -29,6 +29,7 @@ struct WsLayout {
   size_t qbar;        // f32 [h_q][N_b][d]
   size_t kbar;        // f32 [h_kv][N_b][d]
   size_t tri;         // f32 [h_q][N_b(N_b+1)/2]  normalised pooled map, row-major triangle
+  size_t tri_stats;   // f32x4 [h_q][N_b][ceil(N_b/64)] (max, sum of 2^(l - max), min, 0) of each row's 64-column tiles
   size_t hist;        // per head: PeHist
   size_t pe_state;    // per head: PeState
   size_t tie_rows;    // u32 [h_q][N_b] ties per row, then exclusive offsets

@@ -26,6 +26,8 @@ struct PeArgs {
   float* qbar;
   float* kbar;
   float* tri_buf;
+  float4* tri_stats;   // [h_q][nb][n_ct] per-tile row (max, sum of 2^(l - max), min, 0)
+  int n_ct;            // 64-column tiles per row
   PeHist* hist;
   PeState* state;
   uint32_t* tie_rows;
@@ -39,6 +41,10 @@ __device__ __forceinline__ long long tri_off(int r) { return (long long)r * (r +
 
 __device__ __forceinline__ float warp_max(float v) {
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_min(float v) {
+  for (int o = 16; o > 0; o >>= 1) v = fminf(v, __shfl_xor_sync(0xffffffffu, v, o));
   return v;
 }
 __device__ __forceinline__ float warp_sum(float v) {
@@ -151,10 +157,36 @@ __global__ void __launch_bounds__(256) pe_logits_kernel(PeArgs a) {
 #pragma unroll
       for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(qa[i], ka[j], acc[i][j]);
   }
+  // the row statistics of this tile's 64 columns: max, sum of 2^(l - max)
+  // and min over the kept columns c <= r (the 16 threads of a row reduce by
+  // shuffles)
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int r = r0 + ty * 4 + i;
+    float m = -INFINITY, mn = INFINITY;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int c = c0 + tx * 4 + j;
+      if (c <= r) {
+        m = fmaxf(m, acc[i][j]);
+        mn = fminf(mn, acc[i][j]);
+      }
+    }
+#pragma unroll
+    for (int o = 1; o < 16; o <<= 1) {
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    }
+    float sum = 0.f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int c = c0 + tx * 4 + j;
+      if (c <= r) sum += dev::ex2(acc[i][j] - m);
+    }
+#pragma unroll
+    for (int o = 1; o < 16; o <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
     if (r >= a.nb) continue;
+    if (tx == 0) a.tri_stats[((size_t)h * a.nb + r) * a.n_ct + ct] = make_float4(m, sum, mn, 0.f);
     float* row = a.tri_buf + (size_t)h * a.tri_stride + tri_off(r);
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -175,40 +207,69 @@ constexpr int kRowsPerCta = 8;  // one warp per row
 // normalised map is at most 1 / N_b, so its bucket is below 0x3F8.
 constexpr int kL0Low = 1024;
 
+constexpr int kWin = 64;   // level-0 buckets of a row's window in the per-warp histogram
+
 // Row softmax of the pooled logits, divided by N_b (the flattened map's
 // total), written in place; level-0 histogram (bits 31..20) with float64
-// mass. One warp per row. Each lane merges runs of equal buckets, the CTA
-// gathers counts and mass in a shared-memory histogram of all level-0
-// buckets below 1.0, and the non-empty buckets reach the global histogram
-// with one atomic each.
+// mass. One warp per row; the row maximum and normaliser come from the
+// logits kernel's per-tile statistics, so the row is read once. Each lane
+// merges runs of equal buckets; a row whose values span fewer than kWin
+// buckets gathers them in its warp's own window (lanes of one warp mostly
+// hit one bucket, so windows keep contention inside a warp), a wider row
+// (a heavy-tailed map) in the CTA's histogram of all level-0 buckets below
+// 1.0. Non-empty buckets reach the global histogram with one atomic each.
 __global__ void __launch_bounds__(256) pe_softmax_kernel(PeArgs a) {
   const int h = blockIdx.y;
   if (a.route[h] != 1) return;   // uniform over the CTA
   __shared__ unsigned long long scount[kL0Low];
   __shared__ double smass[kL0Low];
+  __shared__ unsigned long long wcount[kRowsPerCta][kWin];
+  __shared__ double wmass[kRowsPerCta][kWin];
   for (int i = threadIdx.x; i < kL0Low; i += blockDim.x) {
     scount[i] = 0;
     smass[i] = 0.0;
   }
-  __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = lane; i < kWin; i += 32) {
+    wcount[warp][i] = 0;
+    wmass[warp][i] = 0.0;
+  }
+  __syncthreads();
   const int r = blockIdx.x * kRowsPerCta + warp;
   PeHist* hist = a.hist + h;
+  uint32_t b_lo = 0;
+  bool window = false;
   if (r < a.nb) {
     float* row = a.tri_buf + (size_t)h * a.tri_stride + tri_off(r);
-    float m = -INFINITY;
-    for (int c = lane; c <= r; c += 32) m = fmaxf(m, row[c]);
+    // row maximum and normaliser from the logits kernel's per-tile statistics
+    const float4* st = a.tri_stats + ((size_t)h * a.nb + r) * a.n_ct;
+    const int n_t = r / kLT + 1;   // column tiles holding c <= r
+    float m = -INFINITY, mn = INFINITY;
+    for (int i = lane; i < n_t; i += 32) {
+      m = fmaxf(m, st[i].x);
+      mn = fminf(mn, st[i].z);
+    }
     m = warp_max(m);
+    mn = warp_min(mn);
     float s = 0.f;
-    for (int c = lane; c <= r; c += 32) s += dev::ex2(row[c] - m);
+    for (int i = lane; i < n_t; i += 32) {
+      const float4 e = st[i];
+      s += e.y * dev::ex2(e.x - m);
+    }
     s = warp_sum(s);
     const float inv = 1.f / (s * (float)a.nb);
+    const uint32_t b_hi = __float_as_uint(inv) >> 20;                       // bucket of the row maximum
+    b_lo = __float_as_uint(dev::ex2(mn - m) * inv) >> 20;                   // bucket of the row minimum
+    window = b_hi >= b_lo && b_hi - b_lo < (uint32_t)kWin;
     uint32_t cur = 0xffffffffu;
     unsigned long long cnt = 0;
     double mass = 0.0;
     auto flush = [&]() {
       if (!cnt) return;
-      if (cur < (uint32_t)kL0Low) {
+      if (window) {
+        atomicAdd(&wcount[warp][cur - b_lo], cnt);
+        atomicAdd(&wmass[warp][cur - b_lo], mass);
+      } else if (cur < (uint32_t)kL0Low) {
         atomicAdd(&scount[cur], cnt);
         atomicAdd(&smass[cur], mass);
       } else {
@@ -231,6 +292,10 @@ __global__ void __launch_bounds__(256) pe_softmax_kernel(PeArgs a) {
     flush();
   }
   __syncthreads();
+  if (window) {   // the warp's window into the global histogram
+    for (int i = lane; i < kWin; i += 32)
+      if (wcount[warp][i]) hist_flush(hist, b_lo + (uint32_t)i, wcount[warp][i], wmass[warp][i]);
+  }
   for (int i = threadIdx.x; i < kL0Low; i += blockDim.x)
     if (scount[i]) hist_flush(hist, (uint32_t)i, scount[i], smass[i]);
 }
@@ -501,6 +566,8 @@ cudaError_t launch_pe(const void* q, const void* k, const Shape& s, char* ws, co
   a.qbar = reinterpret_cast<float*>(ws + L.qbar);
   a.kbar = reinterpret_cast<float*>(ws + L.kbar);
   a.tri_buf = reinterpret_cast<float*>(ws + L.tri);
+  a.tri_stats = reinterpret_cast<float4*>(ws + L.tri_stats);
+  a.n_ct = (s.nb + kLT - 1) / kLT;
   a.hist = reinterpret_cast<PeHist*>(ws + L.hist);
   a.state = reinterpret_cast<PeState*>(ws + L.pe_state);
   a.tie_rows = reinterpret_cast<uint32_t*>(ws + L.tie_rows);
