@@ -165,6 +165,26 @@ crisp_status crisp_prefill_varlen(const void* const* q, const void* const* k, co
                                   void* const* out, const int32_t* n, int32_t count,
                                   const crisp_cfg* cfg, void* stream);
 
+/* Algorithm 1 on a layer held in HOST memory (no counterpart in the paper).
+ * q and out are host [h_q][n][d], k and v host [h_kv][n][d]; they should be
+ * page-locked (cudaHostAlloc / cudaHostRegister) or the copies do not
+ * overlap. The layer runs one KV group at a time (its h_q/h_kv query heads
+ * and one K/V head, the same arithmetic as crisp_prefill on the whole layer):
+ * while group g is computed on `stream`, group g+1 is copied in and group
+ * g-1's output copied out on `copy_stream` (a different stream), with
+ * events ordering the two. cfg describes the whole layer; cfg->workspace
+ * must hold crisp_workspace_size_host(cfg) bytes (one group's scratch, whose
+ * status word crisp_device_status reads as usual, then device copies of two
+ * groups' Q, K, V and out). The call returns once
+ * everything is enqueued; when `stream` completes, out holds the result, so
+ * the host buffers must stay valid until then. copy_stream == stream:
+ * CRISP_ERR_INVALID_ARG. */
+crisp_status crisp_prefill_host(const void* q, const void* k, const void* v, void* out,
+                                const crisp_cfg* cfg, void* stream, void* copy_stream);
+
+/* Workspace bytes crisp_prefill_host needs for cfg's layer. */
+crisp_status crisp_workspace_size_host(const crisp_cfg* cfg, size_t* bytes);
+
 /* Exact dense causal attention with the same kernels (the speed reference). */
 crisp_status crisp_dense_attention(const void* q, const void* k, const void* v, void* out,
                                    const crisp_cfg* cfg, void* stream);

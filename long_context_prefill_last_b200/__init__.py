@@ -34,7 +34,8 @@ STATUS_NAMES = {
 SYMBOLS = ["crisp_cfg_init", "crisp_workspace_size", "crisp_index_dims", "crisp_route", "crisp_select",
            "crisp_attend", "crisp_prefill", "crisp_dense_attention", "crisp_device_status",
            "crisp_status_string", "crisp_version", "crisp_route_noalloc", "crisp_exp2_selftest",
-           "crisp_prefill_batch", "crisp_workspace_size_batch", "crisp_prefill_varlen"]
+           "crisp_prefill_batch", "crisp_workspace_size_batch", "crisp_prefill_varlen",
+           "crisp_prefill_host", "crisp_workspace_size_host"]
 
 
 def library_path() -> str:
@@ -89,6 +90,8 @@ def lib() -> ctypes.CDLL:
         L.crisp_attend.argtypes = [vp, vp, vp, vp, cfgp, ctypes.POINTER(_Index), vp]
         L.crisp_prefill.argtypes = [vp, vp, vp, vp, cfgp, vp]
         L.crisp_prefill_batch.argtypes = [vp, vp, vp, vp, cfgp, ctypes.c_int32, vp]
+        L.crisp_prefill_host.argtypes = [vp, vp, vp, vp, cfgp, vp, vp]
+        L.crisp_workspace_size_host.argtypes = [cfgp, ctypes.POINTER(ctypes.c_size_t)]
         L.crisp_workspace_size_batch.argtypes = [cfgp, ctypes.c_int32, ctypes.POINTER(ctypes.c_size_t)]
         L.crisp_prefill_varlen.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.POINTER(vp),
                                            ctypes.POINTER(vp), ctypes.POINTER(ctypes.c_int32), ctypes.c_int32,
@@ -153,12 +156,16 @@ class Config:
             c.workspace_bytes = self.workspace.numel() * self.workspace.element_size()
         return c
 
-    def allocate_workspace(self, device="cuda", batch: int = 1, max_n: Optional[int] = None):
-        """Device workspace for this shape; `batch` sequences (crisp_prefill_batch)
-        or sequences up to `max_n` tokens (crisp_prefill_varlen)."""
+    def allocate_workspace(self, device="cuda", batch: int = 1, max_n: Optional[int] = None, host: bool = False):
+        """Device workspace for this shape; `batch` sequences (crisp_prefill_batch),
+        sequences up to `max_n` tokens (crisp_prefill_varlen) or a layer in host
+        memory (crisp_prefill_host)."""
         import torch
         c = dataclasses.replace(self, n=max_n) if max_n is not None else self
-        nbytes = workspace_size(c) if batch == 1 else workspace_size_batch(c, batch)
+        if host:
+            nbytes = workspace_size_host(c)
+        else:
+            nbytes = workspace_size(c) if batch == 1 else workspace_size_batch(c, batch)
         self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=device)
         return self.workspace
 
@@ -173,6 +180,12 @@ def workspace_size_batch(cfg: Config, batch: int) -> int:
     out = ctypes.c_size_t(0)
     _check(lib().crisp_workspace_size_batch(ctypes.byref(cfg._c()), int(batch), ctypes.byref(out)),
            "crisp_workspace_size_batch")
+    return out.value
+
+
+def workspace_size_host(cfg: Config) -> int:
+    out = ctypes.c_size_t(0)
+    _check(lib().crisp_workspace_size_host(ctypes.byref(cfg._c()), ctypes.byref(out)), "crisp_workspace_size_host")
     return out.value
 
 
@@ -254,6 +267,23 @@ def prefill_batch(q, k, v, out, cfg: Config, stream=None) -> None:
     """crisp_prefill_batch: q/out [batch, h_q, n, d], k/v [batch, h_kv, n, d]; cfg is one sequence's."""
     _check(lib().crisp_prefill_batch(_ptr(q), _ptr(k), _ptr(v), _ptr(out), ctypes.byref(cfg._c()), int(q.shape[0]),
                                      _stream(stream)), "crisp_prefill_batch")
+
+
+_COPY_STREAMS = {}
+
+
+def prefill_host(q, k, v, out, cfg: Config, stream=None, copy_stream=None) -> None:
+    """crisp_prefill_host: q/out [h_q, n, d] and k/v [h_kv, n, d] in page-locked
+    host memory; copies run on `copy_stream` (one per device by default) and
+    overlap the kernels on `stream`. Completes with `stream`."""
+    import torch
+    if copy_stream is None:
+        dev = torch.cuda.current_device()
+        if dev not in _COPY_STREAMS:
+            _COPY_STREAMS[dev] = torch.cuda.Stream(device=dev)
+        copy_stream = _COPY_STREAMS[dev]
+    _check(lib().crisp_prefill_host(_ptr(q), _ptr(k), _ptr(v), _ptr(out), ctypes.byref(cfg._c()), _stream(stream),
+                                    _stream(copy_stream)), "crisp_prefill_host")
 
 
 def prefill_varlen(qs, ks, vs, outs, cfg: Config, stream=None) -> None:

@@ -240,6 +240,36 @@ static crisp_status fold_batch(const crisp_cfg* cfg, int32_t batch, crisp_cfg* f
   return CRISP_OK;
 }
 
+// Device staging of crisp_prefill_host: one group's scratch workspace first
+// (so the status word sits at offset 0, where crisp_device_status reads it),
+// then two slots of one KV group's Q, K, V and out.
+struct HostPlan {
+  crisp_cfg group_cfg;       // one KV group: h_q / h_kv query heads, one K/V head
+  size_t q_bytes, kv_bytes;  // per group
+  size_t slot_bytes;         // Q + K + V + out of one group, 256-byte aligned pieces
+  size_t slot_off, total;
+};
+
+static crisp_status host_plan(const crisp_cfg* cfg, HostPlan* p) {
+  Shape s;
+  crisp_status r = make_shape(cfg, &s);
+  if (r != CRISP_OK) return r;
+  p->group_cfg = *cfg;
+  p->group_cfg.h_q = s.group;
+  p->group_cfg.h_kv = 1;
+  p->group_cfg.workspace = nullptr;
+  p->group_cfg.workspace_bytes = 0;
+  Shape gs;
+  if ((r = make_shape(&p->group_cfg, &gs)) != CRISP_OK) return r;
+  const size_t elem = s.fp32 ? 4 : 2;
+  p->q_bytes = (size_t)s.group * s.n * s.d * elem;
+  p->kv_bytes = (size_t)s.n * s.d * elem;
+  p->slot_bytes = 2 * align256(p->q_bytes) + 2 * align256(p->kv_bytes);
+  p->slot_off = align256(ws_layout(gs).total);
+  p->total = p->slot_off + 2 * p->slot_bytes;
+  return CRISP_OK;
+}
+
 }  // namespace crisp
 
 using namespace crisp;
@@ -349,6 +379,102 @@ crisp_status crisp_prefill_batch(const void* q, const void* k, const void* v, vo
   return prefill_impl(q, k, v, out, &f, static_cast<cudaStream_t>(stream), true);
 }
 
+crisp_status crisp_workspace_size_host(const crisp_cfg* cfg, size_t* bytes) {
+  HostPlan p;
+  crisp_status r = host_plan(cfg, &p);
+  if (r != CRISP_OK) return r;
+  if (bytes == nullptr) return CRISP_ERR_INVALID_ARG;
+  *bytes = p.total;
+  return CRISP_OK;
+}
+
+crisp_status crisp_prefill_host(const void* q, const void* k, const void* v, void* out, const crisp_cfg* cfg,
+                                void* stream, void* copy_stream) {
+  HostPlan p;
+  crisp_status r = host_plan(cfg, &p);
+  if (r != CRISP_OK) return r;
+  const void* hp[] = {q, k, v, out};
+  for (const void* x : hp)
+    if ((r = check_tensor(x)) != CRISP_OK) return r;
+  if (cfg->workspace == nullptr) return CRISP_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(cfg->workspace) % 256 != 0) return CRISP_ERR_ALIGN;
+  if (cfg->workspace_bytes < p.total) return CRISP_ERR_WORKSPACE;
+  if (copy_stream == stream) return CRISP_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream), cs = static_cast<cudaStream_t>(copy_stream);
+  char* ws = static_cast<char*>(cfg->workspace);
+  crisp_cfg gc = p.group_cfg;
+  gc.workspace = ws;
+  gc.workspace_bytes = p.slot_off;
+  const int n_groups = cfg->h_kv;
+  char* slot_q[2];
+  char* slot_k[2];
+  char* slot_v[2];
+  char* slot_o[2];
+  for (int b = 0; b < 2; ++b) {
+    char* base = ws + p.slot_off + b * p.slot_bytes;
+    slot_q[b] = base;
+    slot_k[b] = base + align256(p.q_bytes);
+    slot_v[b] = slot_k[b] + align256(p.kv_bytes);
+    slot_o[b] = slot_v[b] + align256(p.kv_bytes);
+  }
+  // events: group copied in, group computed; one more for the last copy out
+  cudaEvent_t ev[2 * 64 + 1];
+  const int n_ev = 2 * n_groups + 1;
+  if (n_groups > 64) return CRISP_ERR_UNSUPPORTED;
+  for (int i = 0; i < n_ev; ++i) {
+    if (cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming) != cudaSuccess) {
+      for (int j = 0; j < i; ++j) cudaEventDestroy(ev[j]);
+      return CRISP_ERR_CUDA;
+    }
+  }
+  cudaEvent_t* ev_in = ev;
+  cudaEvent_t* ev_done = ev + n_groups;
+  cudaEvent_t ev_last = ev[2 * n_groups];
+  auto h2d = [&](int g) -> cudaError_t {
+    const int b = g & 1;
+    cudaError_t e;
+    if ((e = cudaMemcpyAsync(slot_q[b], static_cast<const char*>(q) + g * p.q_bytes, p.q_bytes,
+                             cudaMemcpyHostToDevice, cs)) != cudaSuccess)
+      return e;
+    if ((e = cudaMemcpyAsync(slot_k[b], static_cast<const char*>(k) + g * p.kv_bytes, p.kv_bytes,
+                             cudaMemcpyHostToDevice, cs)) != cudaSuccess)
+      return e;
+    if ((e = cudaMemcpyAsync(slot_v[b], static_cast<const char*>(v) + g * p.kv_bytes, p.kv_bytes,
+                             cudaMemcpyHostToDevice, cs)) != cudaSuccess)
+      return e;
+    return cudaEventRecord(ev_in[g], cs);
+  };
+  auto d2h = [&](int g) -> cudaError_t {
+    cudaError_t e;
+    if ((e = cudaStreamWaitEvent(cs, ev_done[g], 0)) != cudaSuccess) return e;
+    return cudaMemcpyAsync(static_cast<char*>(out) + g * p.q_bytes, slot_o[g & 1], p.q_bytes,
+                           cudaMemcpyDeviceToHost, cs);
+  };
+  // the copy stream must not start before work the caller queued on `stream`
+  // (e.g. producing the host buffers' consumers) is ordered: start both
+  // streams from the same point
+  cudaError_t e = cudaEventRecord(ev_last, st);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(cs, ev_last, 0);
+  for (int g = 0; g < n_groups && e == cudaSuccess && r == CRISP_OK; ++g) {
+    // copy stream: group g in (its slot was emptied by group g-2's copy out)
+    if (g >= 2 && (e = d2h(g - 2)) != cudaSuccess) break;
+    if (g < 2 && (e = h2d(g)) != cudaSuccess) break;
+    if (g >= 2 && (e = h2d(g)) != cudaSuccess) break;
+    // compute stream: group g once it is in
+    if ((e = cudaStreamWaitEvent(st, ev_in[g], 0)) != cudaSuccess) break;
+    const int b = g & 1;
+    r = prefill_impl(slot_q[b], slot_k[b], slot_v[b], slot_o[b], &gc, st, g == 0);
+    if (r == CRISP_OK) e = cudaEventRecord(ev_done[g], st);
+  }
+  // the last two groups' outputs, then `stream` waits for the copy stream
+  for (int g = std::max(0, n_groups - 2); g < n_groups && e == cudaSuccess && r == CRISP_OK; ++g) e = d2h(g);
+  if (e == cudaSuccess && r == CRISP_OK) e = cudaEventRecord(ev_last, cs);
+  if (e == cudaSuccess && r == CRISP_OK) e = cudaStreamWaitEvent(st, ev_last, 0);
+  for (int i = 0; i < n_ev; ++i) cudaEventDestroy(ev[i]);
+  if (r != CRISP_OK) return r;
+  return e == cudaSuccess ? CRISP_OK : CRISP_ERR_CUDA;
+}
+
 crisp_status crisp_prefill_varlen(const void* const* q, const void* const* k, const void* const* v,
                                   void* const* out, const int32_t* n, int32_t count, const crisp_cfg* cfg,
                                   void* stream) {
@@ -392,8 +518,11 @@ crisp_status crisp_device_status(const crisp_cfg* cfg, void* stream, int32_t* de
   crisp_status r = make_shape(cfg, &s);
   if (r != CRISP_OK) return r;
   if (device_status == nullptr) return CRISP_ERR_INVALID_ARG;
-  WsLayout L = ws_layout(s);
-  if ((r = check_ws(cfg, L)) != CRISP_OK) return r;
+  // only the status word (the first 32 bytes of every workspace layout) is read
+  if (cfg->workspace == nullptr) return CRISP_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(cfg->workspace) % 256 != 0) return CRISP_ERR_ALIGN;
+  if (cfg->workspace_bytes < 256) return CRISP_ERR_WORKSPACE;
+  const WsLayout L = ws_layout(s);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(cfg->workspace);
   int32_t word[2] = {0, 0};

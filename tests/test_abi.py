@@ -184,3 +184,22 @@ def test_batch_and_varlen_validation_before_any_launch():
     small = crisp.Config(n=2048, h_q=8, h_kv=2)
     small.workspace = _FakeTensor(0x100000, crisp.workspace_size(small))  # too small for n=4096
     assert fn(q, k, v, o, n_ok, 2, ctypes.byref(small._c()), None) == 5
+
+
+def test_host_prefill_workspace_and_validation_before_any_launch():
+    L = crisp.lib()
+    cfg = crisp.Config(n=4096, h_q=8, h_kv=2)
+    group = crisp.Config(n=4096, h_q=4, h_kv=1)
+    per_group = lambda nbytes: (nbytes + 255) // 256 * 256
+    q_bytes, kv_bytes = 4 * 4096 * 128 * 2, 4096 * 128 * 2
+    slots = 2 * (2 * per_group(q_bytes) + 2 * per_group(kv_bytes))
+    assert crisp.workspace_size_host(cfg) == per_group(crisp.workspace_size(group)) + slots
+    c = cfg._c()
+    # no workspace, null host buffer, misaligned host buffer, same stream twice
+    assert L.crisp_prefill_host(0x10000, 0x20000, 0x30000, 0x40000, ctypes.byref(c), None, 0x1) == 5
+    assert L.crisp_prefill_host(0, 0x20000, 0x30000, 0x40000, ctypes.byref(c), None, 0x1) == 1
+    assert L.crisp_prefill_host(0x10004, 0x20000, 0x30000, 0x40000, ctypes.byref(c), None, 0x1) == 4
+    cfg.workspace = _FakeTensor(0x100000, crisp.workspace_size_host(cfg))
+    assert L.crisp_prefill_host(0x10000, 0x20000, 0x30000, 0x40000, ctypes.byref(cfg._c()), 0x7, 0x7) == 1
+    cfg.workspace = _FakeTensor(0x100000, crisp.workspace_size_host(cfg) - 256)
+    assert L.crisp_prefill_host(0x10000, 0x20000, 0x30000, 0x40000, ctypes.byref(cfg._c()), None, 0x1) == 5

@@ -306,6 +306,26 @@ def test_batch_and_varlen_match_single_calls():
     assert torch.equal(outs[0], singles[2]) and torch.equal(outs[1], singles[0]) and torch.equal(outs[2], singles[1])
 
 
+def test_host_prefill_matches_device_prefill():
+    # the layer in page-locked host memory, computed KV group by KV group with
+    # the copies on a second stream: the same output as the device call
+    layer = S.generate(S.scaled("B", n=4096, h_q=16, h_kv=4))
+    qh, kh, vh = (t.pin_memory() for t in S.to_torch(layer))
+    q, k, v = qh.cuda(), kh.cuda(), vh.cuda()
+    cfg = make_cfg(layer)
+    ref = torch.empty_like(q)
+    crisp.prefill(q, k, v, ref, cfg)
+    crisp.raise_on_device_status(cfg)
+    c = layer.cfg
+    hcfg = crisp.Config(n=c.n, h_q=c.h_q, h_kv=c.h_kv, d=c.d, dtype=crisp.BF16)
+    hcfg.allocate_workspace(host=True)
+    out_h = torch.empty(qh.shape, dtype=qh.dtype).pin_memory()
+    crisp.prefill_host(qh, kh, vh, out_h, hcfg)
+    torch.cuda.current_stream().synchronize()
+    crisp.raise_on_device_status(hcfg, where="prefill_host")
+    assert torch.equal(out_h, ref.cpu())
+
+
 # ----------------------------------------------------------------------------- full-size layers
 
 @pytest.mark.parametrize("name", ["B", "C", "D", "E", "E_cliff"])
