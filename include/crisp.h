@@ -227,6 +227,14 @@ crisp_status crisp_route_noalloc(const void* q, const void* k, const crisp_cfg* 
  * (device pointers; poly3, poly5 and ref receive n values each). */
 crisp_status crisp_exp2_selftest(const float* x, float* poly3, float* poly5, float* ref, int32_t n, void* stream);
 
+/* Diagnostics: run the bounded mbarrier wait every kernel uses against a
+ * barrier nothing arrives on, giving up after limit_cycles SM clocks
+ * (1000 <= limit_cycles <= 4e9). status points to 8 int32 of device memory
+ * laid out like the workspace status word (zeroed by the caller); after the
+ * stream completes it holds CRISP_ERR_TIMEOUT and the wait site 99. Checks
+ * that a wait which runs out ends the kernel with a status, not a hang. */
+crisp_status crisp_wait_selftest(int64_t limit_cycles, int32_t* status, void* stream);
+
 /* Library version as major*10000 + minor*100 + patch. */
 int32_t crisp_version(void);
 

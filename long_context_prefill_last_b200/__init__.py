@@ -35,7 +35,7 @@ SYMBOLS = ["crisp_cfg_init", "crisp_workspace_size", "crisp_index_dims", "crisp_
            "crisp_attend", "crisp_prefill", "crisp_dense_attention", "crisp_device_status",
            "crisp_status_string", "crisp_version", "crisp_route_noalloc", "crisp_exp2_selftest",
            "crisp_prefill_batch", "crisp_workspace_size_batch", "crisp_prefill_varlen",
-           "crisp_prefill_host", "crisp_workspace_size_host"]
+           "crisp_prefill_host", "crisp_workspace_size_host", "crisp_wait_selftest"]
 
 
 def library_path() -> str:
@@ -86,6 +86,7 @@ def lib() -> ctypes.CDLL:
         L.crisp_route.argtypes = [vp, vp, cfgp, vp, vp, vp]
         L.crisp_route_noalloc.argtypes = [vp, vp, cfgp, vp, vp, vp]
         L.crisp_exp2_selftest.argtypes = [vp, vp, vp, vp, ctypes.c_int32, vp]
+        L.crisp_wait_selftest.argtypes = [ctypes.c_int64, vp, vp]
         L.crisp_select.argtypes = [vp, vp, cfgp, ctypes.POINTER(_Index), vp]
         L.crisp_attend.argtypes = [vp, vp, vp, vp, cfgp, ctypes.POINTER(_Index), vp]
         L.crisp_prefill.argtypes = [vp, vp, vp, vp, cfgp, vp]
@@ -310,6 +311,12 @@ def exp2_selftest(x, stream=None):
     _check(lib().crisp_exp2_selftest(_ptr(x), _ptr(outs[0]), _ptr(outs[1]), _ptr(outs[2]), x.numel(),
                                      _stream(stream)), "crisp_exp2_selftest")
     return tuple(outs)
+
+
+def wait_selftest(limit_cycles: int, status, stream=None) -> None:
+    """Run the bounded mbarrier wait against a barrier nothing arrives on;
+    `status` (int32[8] CUDA tensor, zeroed) receives CRISP_ERR_TIMEOUT and site 99."""
+    _check(lib().crisp_wait_selftest(int(limit_cycles), _ptr(status), _stream(stream)), "crisp_wait_selftest")
 
 
 def device_status(cfg: Config, stream=None) -> int:

@@ -64,7 +64,7 @@ constexpr long long kWaitLimitCycles = 1000000000LL;
 // the CTA abort flag and the global status) if the wait ran out, or if the
 // abort flag or the global status was already set.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          int32_t* gstatus, int where) {
+                                          int32_t* gstatus, int where, long long limit = kWaitLimitCycles) {
   if (mbar_try_wait(bar, parity)) return true;
   long long t0 = clock64();
   for (uint32_t it = 1;; ++it) {
@@ -75,7 +75,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
         *abort_flag = 1;
         return false;
       }
-      if (clock64() - t0 > kWaitLimitCycles) {
+      if (clock64() - t0 > limit) {
         *abort_flag = 1;
         report(gstatus, CRISP_ERR_TIMEOUT, where);
         return false;

@@ -203,3 +203,10 @@ def test_host_prefill_workspace_and_validation_before_any_launch():
     assert L.crisp_prefill_host(0x10000, 0x20000, 0x30000, 0x40000, ctypes.byref(cfg._c()), 0x7, 0x7) == 1
     cfg.workspace = _FakeTensor(0x100000, crisp.workspace_size_host(cfg) - 256)
     assert L.crisp_prefill_host(0x10000, 0x20000, 0x30000, 0x40000, ctypes.byref(cfg._c()), None, 0x1) == 5
+
+
+def test_wait_selftest_validates_before_launch():
+    L = crisp.lib()
+    assert L.crisp_wait_selftest(10, 0x10000, None) == 1          # limit below 1000 cycles
+    assert L.crisp_wait_selftest(5_000_000_000, 0x10000, None) == 1
+    assert L.crisp_wait_selftest(1_000_000, 0, None) == 1         # no status buffer

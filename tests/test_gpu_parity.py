@@ -326,6 +326,36 @@ def test_host_prefill_matches_device_prefill():
     assert torch.equal(out_h, ref.cpu())
 
 
+def test_bounded_wait_runs_out_with_a_status_and_the_context_survives():
+    # the wait every kernel uses, on a barrier nothing arrives on, with a
+    # limit of about a millisecond: the kernel ends and reports the site
+    st = torch.zeros(8, dtype=torch.int32, device="cuda")
+    crisp.wait_selftest(2_000_000, st)
+    torch.cuda.synchronize()
+    assert int(st[0]) == 9 and int(st[1]) == 99          # CRISP_ERR_TIMEOUT at site 99
+    layer = S.generate(S.scaled("B", n=1024, h_q=4, h_kv=2))
+    q, k, v = device_layer(layer)
+    cfg = make_cfg(layer)
+    out = torch.empty_like(q)
+    crisp.prefill(q, k, v, out, cfg)
+    crisp.raise_on_device_status(cfg)
+    assert torch.isfinite(out.float()).all()
+
+
+def test_nonfinite_proxy_statistics_are_reported_not_trapped():
+    layer = S.generate(S.scaled("B", n=2048, h_q=4, h_kv=2))
+    q, k, v = device_layer(layer)
+    cfg = make_cfg(layer)
+    bad = q.clone()
+    bad[1, -1, :] = float("nan")                          # a proxy row of query head 1
+    out = torch.empty_like(q)
+    crisp.prefill(bad, k, v, out, cfg)
+    assert crisp.device_status(cfg) == 10                  # CRISP_ERR_NONFINITE (and cleared by the read)
+    crisp.prefill(q, k, v, out, cfg)                       # the next call runs normally
+    crisp.raise_on_device_status(cfg)
+    assert torch.isfinite(out.float()).all()
+
+
 # ----------------------------------------------------------------------------- full-size layers
 
 @pytest.mark.parametrize("name", ["B", "C", "D", "E", "E_cliff"])
