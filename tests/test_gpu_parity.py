@@ -160,6 +160,9 @@ SMALL = {
     "B-4k-gamma0.5": (lambda: S.scaled("B", n=4096, h_q=8, h_kv=2), {"gamma": 0.5}),
     "B-4k-forcePE": (lambda: S.scaled("B", n=4096, h_q=8, h_kv=2), {"force_route": 1}),
     "B-4k-alphaHuge": (lambda: S.scaled("B", n=4096, h_q=8, h_kv=2), {"alpha": 1e30}),
+    # the largest KV group the kernels take (16 query heads per K/V head): all VS, all PE
+    "B-2k-group16-VS": (lambda: S.scaled("B", n=2048, h_q=16, h_kv=1, planted_groups=[0]), {}),
+    "B-2k-group16-PE": (lambda: S.scaled("B", n=2048, h_q=16, h_kv=1, planted_groups=[]), {"force_route": 1}),
     # mass-cliff background (log-normal block masses): sparser VS and PE selections
     "Ccliff-4k": (lambda: S.scaled("C_cliff", n=4096, h_q=8, h_kv=2), {}),
     "Ccliff-16k": (lambda: S.scaled("C_cliff", n=16384, h_q=8, h_kv=2), {}),
@@ -357,6 +360,27 @@ def test_nonfinite_proxy_statistics_are_reported_not_trapped():
 
 
 # ----------------------------------------------------------------------------- full-size layers
+
+def test_longest_accepted_sequence():
+    # n = 2^20, the largest length the boundary accepts (N_b = 8192, 256 mask
+    # words per row): one planted (VS) and one Gaussian (PE) KV group
+    layer = S.generate(S.scaled("B", n=1 << 20, h_q=8, h_kv=2), threads=16)
+    q, k, v = device_layer(layer)
+    cfg = make_cfg(layer)
+    ocfg = oracle_cfg(cfg)
+    host, _ = gpu_select(q, k, cfg)
+    oidx = oracle_heads(layer, ocfg)
+    rep = P.Report()
+    check_index(host, oidx, cfg, rep)
+    rep.assert_ok()
+    assert all(host["route"][h] == O.VS for h in layer.planted_q_heads)
+    assert all(host["route"][h] == O.PE for h in layer.gaussian_q_heads)
+    out = torch.empty_like(q)
+    crisp.prefill(q, k, v, out, cfg)
+    crisp.raise_on_device_status(cfg, where="prefill")
+    check_outputs(layer, out, oidx, ocfg, sample_rows(cfg.n, cfg.n_blocks, full=False),
+                  skip_heads=rep.heads_with_flips())
+
 
 @pytest.mark.parametrize("name", ["B", "C", "D", "E", "E_cliff"])
 def test_full_size_layer_parity(name):
