@@ -6,6 +6,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <vector>
 
 #include "crisp.h"
 #include "internal.h"
@@ -418,17 +419,16 @@ crisp_status crisp_prefill_host(const void* q, const void* k, const void* v, voi
     slot_o[b] = slot_v[b] + align256(p.kv_bytes);
   }
   // events: group copied in, group computed; one more for the last copy out
-  cudaEvent_t ev[2 * 64 + 1];
   const int n_ev = 2 * n_groups + 1;
-  if (n_groups > 64) return CRISP_ERR_UNSUPPORTED;
+  std::vector<cudaEvent_t> ev(n_ev);
   for (int i = 0; i < n_ev; ++i) {
     if (cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming) != cudaSuccess) {
       for (int j = 0; j < i; ++j) cudaEventDestroy(ev[j]);
       return CRISP_ERR_CUDA;
     }
   }
-  cudaEvent_t* ev_in = ev;
-  cudaEvent_t* ev_done = ev + n_groups;
+  cudaEvent_t* ev_in = ev.data();
+  cudaEvent_t* ev_done = ev.data() + n_groups;
   cudaEvent_t ev_last = ev[2 * n_groups];
   auto h2d = [&](int g) -> cudaError_t {
     const int b = g & 1;
