@@ -112,12 +112,16 @@ __global__ void __launch_bounds__(128) pool_kernel(const T* __restrict__ x, floa
   out[((size_t)head * nb + b) * kHeadDim + tid] = s * (1.f / kBlock);
 }
 
-// Pooled logits (log2 domain) of one 64 x 64 tile (rt, ct), ct <= rt, of the
-// block-causal triangle; thread (ty, tx) holds a 4 x 4 register tile. Both
-// operand tiles sit transposed in shared memory ([d][block], row stride 68
-// floats) so one float4 of each feeds 16 FMAs.
-constexpr int kLT = 64;       // blocks per tile side
-constexpr int kLStride = 68;  // floats per transposed row
+// Pooled logits (log2 domain) of one 128 x 128 tile (rt, ct), ct <= rt, of
+// the block-causal triangle. Thread (ty, tx) holds an 8 x 8 register tile:
+// rows ty*4 + {0..3} and 64 + ty*4 + {0..3}, columns tx*4 + {0..3} and
+// 64 + tx*4 + {0..3}. Both operand tiles sit transposed in shared memory
+// ([d][block], row stride 132 floats), so each step over d reads four float4
+// (contiguous across the threads of a row) for 64 FMAs. The statistics the
+// row softmax needs are kept per 64-column half (kLT).
+constexpr int kLT = 64;        // columns per statistics tile
+constexpr int kLT2 = 128;      // blocks per CTA tile side
+constexpr int kLStride = 132;  // floats per transposed row
 __global__ void __launch_bounds__(256) pe_logits_kernel(PeArgs a) {
   const int h = blockIdx.y;
   if (a.route[h] != 1) return;
@@ -128,12 +132,12 @@ __global__ void __launch_bounds__(256) pe_logits_kernel(PeArgs a) {
   while ((rt + 1) * (rt + 2) / 2 <= ti) ++rt;
   while (rt * (rt + 1) / 2 > ti) --rt;
   const int ct = ti - rt * (rt + 1) / 2;
-  const int r0 = rt * kLT, c0 = ct * kLT;
+  const int r0 = rt * kLT2, c0 = ct * kLT2;
   extern __shared__ __align__(16) float lsm[];
   float* qT = lsm;                        // [128][kLStride]
   float* kT = lsm + kHeadDim * kLStride;  // [128][kLStride]
   const int tid = threadIdx.x;
-  for (int e = tid; e < kLT * kHeadDim; e += 256) {
+  for (int e = tid; e < kLT2 * kHeadDim; e += 256) {
     const int rr = e >> 7, dd = e & 127;
     qT[dd * kLStride + rr] =
         (r0 + rr < a.nb) ? a.qbar[((size_t)h * a.nb + r0 + rr) * kHeadDim + dd] * a.scale_log2 : 0.f;
@@ -141,56 +145,64 @@ __global__ void __launch_bounds__(256) pe_logits_kernel(PeArgs a) {
   }
   __syncthreads();
   const int ty = tid >> 4, tx = tid & 15;
-  float acc[4][4];
+  float acc[8][8];
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+  for (int i = 0; i < 8; ++i)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
-#pragma unroll 4
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+#pragma unroll 2
   for (int dd = 0; dd < kHeadDim; ++dd) {
-    const float4 qv = *reinterpret_cast<const float4*>(qT + dd * kLStride + ty * 4);
-    const float4 kv = *reinterpret_cast<const float4*>(kT + dd * kLStride + tx * 4);
-    const float qa[4] = {qv.x, qv.y, qv.z, qv.w};
-    const float ka[4] = {kv.x, kv.y, kv.z, kv.w};
+    const float* qd = qT + dd * kLStride;
+    const float* kd = kT + dd * kLStride;
+    const float4 q0 = *reinterpret_cast<const float4*>(qd + ty * 4);
+    const float4 q1 = *reinterpret_cast<const float4*>(qd + 64 + ty * 4);
+    const float4 k0 = *reinterpret_cast<const float4*>(kd + tx * 4);
+    const float4 k1 = *reinterpret_cast<const float4*>(kd + 64 + tx * 4);
+    const float qa[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+    const float ka[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < 8; ++i)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(qa[i], ka[j], acc[i][j]);
+      for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(qa[i], ka[j], acc[i][j]);
   }
-  // the row statistics of this tile's 64 columns: max, sum of 2^(l - max)
-  // and min over the kept columns c <= r (the 16 threads of a row reduce by
-  // shuffles)
+  // per row and 64-column half: max, sum of 2^(l - max) and min over the kept
+  // columns c <= r (the 16 threads of a row reduce by shuffles); then the row
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int r = r0 + ty * 4 + i;
-    float m = -INFINITY, mn = INFINITY;
+  for (int i = 0; i < 8; ++i) {
+    const int r = r0 + (i >> 2) * 64 + ty * 4 + (i & 3);
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int c = c0 + tx * 4 + j;
-      if (c <= r) {
-        m = fmaxf(m, acc[i][j]);
-        mn = fminf(mn, acc[i][j]);
+    for (int half = 0; half < 2; ++half) {
+      float m = -INFINITY, mn = INFINITY;
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj) {
+        const int c = c0 + half * 64 + tx * 4 + jj;
+        if (c <= r) {
+          m = fmaxf(m, acc[i][half * 4 + jj]);
+          mn = fminf(mn, acc[i][half * 4 + jj]);
+        }
       }
-    }
 #pragma unroll
-    for (int o = 1; o < 16; o <<= 1) {
-      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-    }
-    float sum = 0.f;
+      for (int o = 1; o < 16; o <<= 1) {
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+      }
+      float sum = 0.f;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int c = c0 + tx * 4 + j;
-      if (c <= r) sum += dev::ex2(acc[i][j] - m);
-    }
+      for (int jj = 0; jj < 4; ++jj) {
+        const int c = c0 + half * 64 + tx * 4 + jj;
+        if (c <= r) sum += dev::ex2(acc[i][half * 4 + jj] - m);
+      }
 #pragma unroll
-    for (int o = 1; o < 16; o <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+      for (int o = 1; o < 16; o <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+      const int c64 = 2 * ct + half;   // statistics tile of this half
+      if (tx == 0 && r < a.nb && c64 * kLT < a.nb && c64 * kLT <= r)
+        a.tri_stats[((size_t)h * a.nb + r) * a.n_ct + c64] = make_float4(m, sum, mn, 0.f);
+    }
     if (r >= a.nb) continue;
-    if (tx == 0) a.tri_stats[((size_t)h * a.nb + r) * a.n_ct + ct] = make_float4(m, sum, mn, 0.f);
     float* row = a.tri_buf + (size_t)h * a.tri_stride + tri_off(r);
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int c = c0 + tx * 4 + j;
+    for (int j = 0; j < 8; ++j) {
+      const int c = c0 + (j >> 2) * 64 + tx * 4 + (j & 3);
       if (c <= r) row[c] = acc[i][j];
     }
   }
@@ -592,7 +604,7 @@ cudaError_t launch_pe(const void* q, const void* k, const Shape& s, char* ws, co
   const size_t lsmem = 2 * kHeadDim * kLStride * sizeof(float);
   e = cudaFuncSetAttribute(pe_logits_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lsmem);
   if (e != cudaSuccess) return e;
-  const int nt = (s.nb + kLT - 1) / kLT;
+  const int nt = (s.nb + kLT2 - 1) / kLT2;
   pe_logits_kernel<<<dim3(nt * (nt + 1) / 2, s.h_q), 256, lsmem, st>>>(a);
   const int row_ctas = (s.nb + kRowsPerCta - 1) / kRowsPerCta;
   pe_softmax_kernel<<<dim3(row_ctas, s.h_q), 256, 0, st>>>(a);
