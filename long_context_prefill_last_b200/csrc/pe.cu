@@ -122,18 +122,15 @@ __global__ void __launch_bounds__(128) pool_kernel(const T* __restrict__ x, floa
 constexpr int kLT = 64;        // columns per statistics tile
 constexpr int kLT2 = 128;      // blocks per CTA tile side
 constexpr int kLStride = 132;  // floats per transposed row
-__global__ void __launch_bounds__(256) pe_logits_kernel(PeArgs a) {
-  const int h = blockIdx.y;
-  if (a.route[h] != 1) return;
+// One tile ti of query head h (routed PE).
+__device__ __forceinline__ void pe_logits_tile(const PeArgs& a, int h, int ti, float* lsm) {
   const int g = h / a.group;
   // linear lower-triangle tile index -> (rt, ct)
-  const int ti = blockIdx.x;
   int rt = (int)((sqrtf(8.f * (float)ti + 1.f) - 1.f) * 0.5f);
   while ((rt + 1) * (rt + 2) / 2 <= ti) ++rt;
   while (rt * (rt + 1) / 2 > ti) --rt;
   const int ct = ti - rt * (rt + 1) / 2;
   const int r0 = rt * kLT2, c0 = ct * kLT2;
-  extern __shared__ __align__(16) float lsm[];
   float* qT = lsm;                        // [128][kLStride]
   float* kT = lsm + kHeadDim * kLStride;  // [128][kLStride]
   const int tid = threadIdx.x;
@@ -205,6 +202,19 @@ __global__ void __launch_bounds__(256) pe_logits_kernel(PeArgs a) {
       const int c = c0 + (j >> 2) * 64 + tx * 4 + (j & 3);
       if (c <= r) row[c] = acc[i][j];
     }
+  }
+}
+
+// A grid-stride loop over (query head, triangle tile) items: heads not
+// routed PE cost one iteration, not a CTA launch (a launched CTA reserves
+// 132 KB of shared memory, one per SM, even when it exits at once).
+__global__ void __launch_bounds__(256) pe_logits_kernel(PeArgs a, int n_tri_tiles) {
+  extern __shared__ __align__(16) float lsm[];
+  for (long long item = blockIdx.x; item < (long long)a.h_q * n_tri_tiles; item += gridDim.x) {
+    const int h = (int)(item / n_tri_tiles);
+    if (a.route[h] != 1) continue;   // uniform over the CTA
+    __syncthreads();                 // the previous item's reads of lsm are done
+    pe_logits_tile(a, h, (int)(item % n_tri_tiles), lsm);
   }
 }
 
@@ -605,7 +615,14 @@ cudaError_t launch_pe(const void* q, const void* k, const Shape& s, char* ws, co
   e = cudaFuncSetAttribute(pe_logits_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lsmem);
   if (e != cudaSuccess) return e;
   const int nt = (s.nb + kLT2 - 1) / kLT2;
-  pe_logits_kernel<<<dim3(nt * (nt + 1) / 2, s.h_q), 256, lsmem, st>>>(a);
+  {
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int n_tri_tiles = nt * (nt + 1) / 2;
+    const long long items = (long long)s.h_q * n_tri_tiles;
+    pe_logits_kernel<<<(int)std::min<long long>(items, sms), 256, lsmem, st>>>(a, n_tri_tiles);
+  }
   const int row_ctas = (s.nb + kRowsPerCta - 1) / kRowsPerCta;
   pe_softmax_kernel<<<dim3(row_ctas, s.h_q), 256, 0, st>>>(a);
   pe_find_kernel<<<s.h_q, 1024, 0, st>>>(a, 0);
