@@ -1,29 +1,42 @@
 """Benchmark: CRISP sparse-prefill attention, ms per layer, and speedup over
 the dense causal attention kernel built the same way, on one B200 per rank.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config E] [--impl crisp|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config E|all] [--impl crisp|reference]
+                    [--alpha A] [--gamma G] [--sweep] [--shard layers|heads]
 
 One step = one pass of the whole hot path over one synthetic layer: proxy map,
 route, VS/PE selection and block-sparse attention (crisp_select then
 crisp_attend, with an event between them so the attention kernel is timed
 live). Inputs stay resident in HBM; they are far larger than L2 at every
-full-size layer, so no flush is needed between steps. The dense reference and
-the end-to-end number (crisp_prefill through host buffers, copies included)
-are timed the same way. With N > 1 (torchrun) every rank runs its own layer
-(weak scaling, no collective on the data path); the step time is the max over
-ranks and the reported ms/layer divides it by N. ``--shard heads`` instead
-splits one layer across the ranks by KV group (strong scaling: each rank draws
-and runs only its groups; the layer's time is the slowest rank's).
+full-size layer, so no flush is needed between steps. Every timed step also
+runs, right after the CRISP step and on the same stream, the dense reference
+(crisp_dense_attention) and the end-to-end call (crisp_prefill_host from
+page-locked host buffers, copies included), so all three are timed over the
+same K steps, interleaved, each with its own CUDA events.
 
-``--impl reference`` times the CPU oracle (float64, host cores) on a bounded
-sample of the same workload and scales it to ms/layer.
+With --gpus N > 1 the script starts N ranks itself (torch.distributed.run,
+one process per GPU) unless it already runs under a launcher. By default
+every rank runs its own layer (weak scaling, no collective on the data path);
+the step time is the max over ranks and the reported ms/layer divides it by
+N. ``--shard heads`` instead splits one layer across the ranks by KV group
+(strong scaling: each rank draws and runs only its groups; the layer's time
+is the slowest rank's).
+
+``--config all`` prints one line per configuration (A-E); ``--sweep`` one
+line per (alpha, gamma) in {1.0, 1.25, 1.5} x {0.95, 0.97} on one layer.
+
+``--impl reference`` times the CPU oracle (float64, host cores): every step
+is a bounded sample of the same workload (the index of one VS and one PE
+head and exact attention on a few query rows of each), scaled to ms/layer.
 """
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import os
+import socket
 import statistics
 import subprocess
 import sys
@@ -40,7 +53,12 @@ import crisp_synth as S  # noqa: E402
 METRIC = "sparse-prefill attention ms/layer & speedup vs in-run dense kernel, 128K–512K"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 PAGES_SPEEDUP_512K = 5.30   # the pages' figure on a single H100 (context only)
-KERNELS_PER_STEP = 17       # proxy 1, finalise 2, VS select 1, PE 12, attention 1
+# kernels of one crisp_select: proxy 1, finalise 2, VS select 1, PE 12
+SELECT_KERNELS = 16
+SWEEP = [(1.0, 0.95), (1.0, 0.97), (1.25, 0.95), (1.25, 0.97), (1.5, 0.95), (1.5, 0.97)]
+ALL_CONFIGS = ["A", "B", "C", "D", "E"]
+# FP32 lanes per SM (the CUDA-core attention of fp32 layers is bound by FFMA issue)
+FP32_LANES_PER_SM = 128
 
 
 def load_peaks():
@@ -88,29 +106,35 @@ class ClockSampler:
             self.proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
-        sm, smax, reasons, power = [], [], set(), []
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                smax.append(float(parts[2]))
-                power.append(float(parts[3]))
-            except ValueError:
-                continue
-            for name, val in zip(("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"),
-                                 parts[5:9]):
-                if val.lower().startswith("active"):
-                    reasons.add(name)
-        loaded = [s for s, p in zip(sm, power) if p > 250] or sm
-        return {"sm_mhz": statistics.median(loaded) if loaded else None,
-                "sm_max_mhz": max(smax) if smax else None,
-                "reasons": sorted(reasons), "samples": len(sm),
-                "power_w_max": max(power) if power else None}
+        return parse_clock_lines(self.lines)
 
 
-# ----------------------------------------------------------------------------- helpers
+def parse_clock_lines(lines):
+    """Median SM clock under load (power above 250 W), max clock and the
+    throttle reasons seen, from nvidia-smi csv lines."""
+    sm, smax, reasons, power = [], [], set(), []
+    for ln in lines:
+        parts = [p.strip() for p in ln.split(",")]
+        if len(parts) < 9:
+            continue
+        try:
+            sm.append(float(parts[1]))
+            smax.append(float(parts[2]))
+            power.append(float(parts[3]))
+        except ValueError:
+            continue
+        for name, val in zip(("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"),
+                             parts[5:9]):
+            if val.lower().startswith("active"):
+                reasons.add(name)
+    loaded = [s for s, p in zip(sm, power) if p > 250] or sm
+    return {"sm_mhz": statistics.median(loaded) if loaded else None,
+            "sm_max_mhz": max(smax) if smax else None,
+            "reasons": sorted(reasons), "samples": len(sm),
+            "power_w_max": max(power) if power else None}
+
+
+# ----------------------------------------------------------------------------- schedule statistics
 
 def unpack_bits(words, nb):
     w = np.ascontiguousarray(words).astype(np.uint32)
@@ -118,27 +142,52 @@ def unpack_bits(words, nb):
     return bits.reshape(*w.shape[:-1], w.shape[-1] * 32)[..., :nb]
 
 
-def kept_tiles(route, vs_mask, pe_mask, nb):
-    """Computed 128x128 tiles of the sparse schedule, summed over heads (the
-    kernel's rule: VS keeps tile (I, t) when column block t or offset block
-    I-t or I-t-1 is selected; PE when block (I, t) is; the diagonal always)."""
-    total = 0
+# (query, key) pairs inside one 128x128 tile of each kind the attention kernel computes
+PAIRS_FULL, PAIRS_LOWER, PAIRS_UPPER = 128 * 128, 128 * 129 // 2, 128 * 127 // 2
+
+
+def schedule_stats(route, vs_mask, pe_mask, nb):
+    """Work of the sparse schedule, summed over heads, by the kernel's rule:
+    VS keeps key tile t of query tile I whole when column block t is selected,
+    the part c <= r when offset block I-t is, the part c > r when offset block
+    I-t-1 is; PE keeps tile (I, t) when block (I, t) is; the diagonal tile
+    (its causal half) always.
+
+    Returns computed 128x128 tiles, selected (query, key) pairs, and the tiles
+    of the union schedules of the query-tile pairs (I, I-1) one CTA computes."""
+    tiles = pairs = union = 0
     I = np.arange(nb)[:, None]
     t = np.arange(nb)[None, :]
     causal = t <= I
+    below = t < I
+    diag = np.arange(nb)
     for h in range(len(route)):
         if route[h] == 1:
-            m = unpack_bits(pe_mask[h], nb) & causal
-            m[np.arange(nb), np.arange(nb)] = True
+            full = unpack_bits(pe_mask[h], nb) & below
+            lower = np.zeros_like(full)
+            upper = np.zeros_like(full)
         else:
             v = unpack_bits(vs_mask[h, 0], nb)
             s = unpack_bits(vs_mask[h, 1], nb)
-            off = np.clip(I - t, 0, nb - 1)
-            off1 = np.clip(I - t - 1, 0, nb - 1)
-            m = causal & (v[t] | s[off] | ((I - t - 1 >= 0) & s[off1]))
-            m[np.arange(nb), np.arange(nb)] = True
-        total += int(m.sum())
-    return total
+            lo = s[np.clip(I - t, 0, nb - 1)] & below
+            hi = s[np.clip(I - t - 1, 0, nb - 1)] & (I - t - 1 >= 0)
+            vcol = v[t] & below
+            full = vcol | (lo & hi)
+            lower = ~full & lo
+            upper = ~full & hi & ~lo
+        kept = full | lower | upper
+        kept[diag, diag] = True
+        tiles += int(kept.sum())
+        pairs += (int(full.sum()) * PAIRS_FULL + int(lower.sum()) * PAIRS_LOWER + int(upper.sum()) * PAIRS_UPPER
+                  + nb * PAIRS_LOWER)
+        # CTA pairs: query tiles (nb-1, nb-2), (nb-3, nb-4), ...; the union over both rows
+        ia = np.arange(nb - 1, -1, -2)
+        ib = ia - 1
+        u = kept[ia].copy()
+        has_b = ib >= 0
+        u[has_b] |= kept[ib[has_b]]
+        union += int(u.sum())
+    return tiles, pairs, union
 
 
 def kernel_source_hash(names):
@@ -149,12 +198,10 @@ def kernel_source_hash(names):
     return h.hexdigest()[:16]
 
 
-# dram__bytes_read.sum + dram__bytes_write.sum of one launch, from the ncu
-# capture summarised in profiles/attn_tc_traffic_layerE.md (layer E, default
-# alpha and gamma); reported only for the kernel source it was taken on.
-MEASURED_TRAFFIC = {
-    ("attn_tc_kernel", "E", 1.0, 0.95): {"source_hash": "e805491e5011c54d", "bytes_per_launch": 949.2e9 + 4.32e9},
-}
+# dram__bytes_read.sum + dram__bytes_write.sum per attention launch, measured
+# by ncu on a scaled case of the layer (one KV group, the same n) and scaled by
+# the KV groups; valid only for the kernel source it was taken on.
+MEASURED_TRAFFIC = {}
 
 
 def load_traffic(kernel, src_hash, config, alpha, gamma):
@@ -185,78 +232,135 @@ def cpu_cores():
         return os.cpu_count() or 1
 
 
+def config_dict(name, alpha, gamma, world=1, heads_mode=False):
+    """The workload description shared by both arms."""
+    c = S.CONFIGS[name]
+    slash_note = ("planted slash offsets dealt round-robin over the planted KV groups "
+                  f"({c.n_slash} per layer, about {max(1, c.n_slash // max(1, len(c.planted_groups)))} per planted "
+                  "group); verticals per planted group as named")
+    return {"workload": f"layer {name}: {c.desc}", "h_q": c.h_q, "h_kv": c.h_kv, "seq_len": c.n,
+            "alpha": alpha, "gamma": gamma, "head_dim": c.d, "batch": 1,
+            "parallelism": (f"one layer split by KV group over {world} GPUs (no exchange)" if heads_mode
+                            else f"independent layer per GPU x{world}"),
+            "structure": slash_note,
+            "l2": ("inputs far exceed the 126 MB L2 at every full-size layer; no flush between steps" if c.n >= 32768
+                   else "small layer: inputs fit in L2 (no flush); timings are launch-bound")}
+
+
 # ----------------------------------------------------------------------------- CPU oracle baseline
 
-def oracle_ms_per_layer(cfg_name: str, budget_s: float = 20.0):
-    """Time the oracle on a bounded sample of the layer and scale to ms/layer.
+class OracleSampler:
+    """The oracle on a bounded sample of a layer, scaled to ms/layer.
 
-    Sample: the proxy/route/selection of one planted (VS) head and one
-    Gaussian (PE) head, and exact sparse attention for sampled query rows of
-    those heads. Scaled: index time per head x heads of each kind; attention
-    time per row x rows x heads (the oracle's attention cost per row grows
-    with the selected keys; rows are drawn evenly over the sequence so their
-    mean matches the layer's)."""
-    from oracle import crisp_oracle as O
-    c = S.CONFIGS[cfg_name]
-    # one KV group of each kind is enough: generate a 2-group slice of the layer
-    small = S.dataclasses.replace(c, h_q=2 * c.group, h_kv=2, planted_groups=(0,),
-                                  slash_groups=len(c.planted_groups) if c.planted_groups else 0)
-    if len(c.planted_groups) == c.h_kv:
-        small = S.dataclasses.replace(small, planted_groups=(0, 1))
-    layer = S.generate(small, threads=8)
-    ocfg = O.OracleCfg()
-    t_index = {}
-    t_rows = {}
-    n = c.n
-    G = c.group
-    t_start = time.perf_counter()
-    heads = {"vs": 0, "pe": G}
-    rows_done = {"vs": 0, "pe": 0}
-    for kind, h in heads.items():
-        q = layer.as_f64("q", h)
-        k = layer.as_f64("k", h // G)
-        v = layer.as_f64("v", h // G)
-        t0 = time.perf_counter()
-        idx = O.head_index(q, k, ocfg)
-        t_index[kind] = time.perf_counter() - t0
-        # attention rows, evenly spread, until this head's share of the budget is used
-        rng = np.random.default_rng(0)
-        t_att = 0.0
-        nrows = 0
-        while t_att < budget_s / 4 and nrows < n:
-            rows = np.sort(rng.choice(n, size=8, replace=False))
+    One sample: the proxy/route/selection of one planted (VS) head and one
+    Gaussian (PE) head, and exact sparse attention for `rows` random query
+    rows of each. Scaled: index time per head x heads of each kind, plus
+    attention time per row x rows x heads (the oracle's attention cost per row
+    grows with the selected keys; rows are drawn uniformly over the sequence,
+    so their mean matches the layer's)."""
+
+    def __init__(self, cfg_name, alpha=1.0, gamma=0.95, threads=8):
+        from oracle import crisp_oracle as O
+        self.O = O
+        c = S.CONFIGS[cfg_name]
+        self.c = c
+        self.name = cfg_name
+        # one KV group of each kind is enough: a 2-group slice of the layer
+        small = dataclasses.replace(c, h_q=2 * c.group, h_kv=2, planted_groups=(0,),
+                                    slash_groups=len(c.planted_groups) if c.planted_groups else 0)
+        if len(c.planted_groups) == c.h_kv:
+            small = dataclasses.replace(small, planted_groups=(0, 1))
+        self.layer = S.generate(small, threads=threads)
+        self.ocfg = O.OracleCfg(alpha=alpha, gamma=gamma)
+        G = c.group
+        self.heads = {"vs": 0, "pe": G} if c.h_q > 1 else {"vs": 0}
+        self.n_vs = len(c.planted_groups) * G
+        self.n_pe = c.h_q - self.n_vs
+        self.rng = np.random.default_rng(0)
+        self.rows_done = {k: 0 for k in self.heads}
+
+    def sample(self, rows=8):
+        """One bounded sample; returns (its wall seconds, the ms/layer it extrapolates to)."""
+        O, c, G = self.O, self.c, self.c.group
+        t_start = time.perf_counter()
+        t_index, t_row = {}, {}
+        for kind, h in self.heads.items():
+            q = self.layer.as_f64("q", h)
+            k = self.layer.as_f64("k", h // G)
+            v = self.layer.as_f64("v", h // G)
             t0 = time.perf_counter()
-            O.head_attention(q, k, v, idx, rows, ocfg, chunk=8)
-            t_att += time.perf_counter() - t0
-            nrows += len(rows)
-        t_rows[kind] = t_att / nrows
-        rows_done[kind] = nrows
-    n_vs = len(c.planted_groups) * G
-    n_pe = c.h_q - n_vs
-    total_s = n_vs * (t_index["vs"] + n * t_rows["vs"]) + n_pe * (t_index["pe"] + n * t_rows["pe"])
-    sample = (f"one planted (VS) and one Gaussian (PE) head of layer {cfg_name}: full proxy/route/selection, "
-              f"exact attention on {rows_done['vs']} + {rows_done['pe']} random query rows; "
-              f"scaled to {c.h_q} heads x {n} rows")
-    return total_s * 1e3, sample, time.perf_counter() - t_start
+            idx = O.head_index(q, k, self.ocfg)
+            t_index[kind] = time.perf_counter() - t0
+            r = np.sort(self.rng.choice(c.n, size=min(rows, c.n), replace=False))
+            t0 = time.perf_counter()
+            O.head_attention(q, k, v, idx, r, self.ocfg, chunk=8)
+            t_row[kind] = (time.perf_counter() - t0) / len(r)
+            self.rows_done[kind] += len(r)
+        if "pe" not in t_index:   # a one-head layer
+            t_index["pe"], t_row["pe"] = t_index["vs"], t_row["vs"]
+        n_vs = self.n_vs if c.h_q > 1 else c.h_q
+        n_pe = self.n_pe if c.h_q > 1 else 0
+        total_s = (n_vs * (t_index["vs"] + c.n * t_row["vs"]) + n_pe * (t_index["pe"] + c.n * t_row["pe"]))
+        return time.perf_counter() - t_start, total_s * 1e3
+
+    def describe(self):
+        parts = " + ".join(str(v) for v in self.rows_done.values())
+        kinds = "one planted (VS) and one Gaussian (PE) head" if len(self.heads) == 2 else "the layer's one head"
+        return (f"{kinds} of layer {self.name}: full proxy/route/selection, exact attention on {parts} random "
+                f"query rows; scaled to {self.c.h_q} heads x {self.c.n} rows")
+
+
+def oracle_ms_per_layer(cfg_name, budget_s=20.0, alpha=1.0, gamma=0.95):
+    """The cpu_baseline leg: samples until about budget_s seconds of CPU work."""
+    smp = OracleSampler(cfg_name, alpha, gamma)
+    est, spent = [], 0.0
+    while spent < budget_s or not est:
+        dt, ms = smp.sample()
+        spent += dt
+        est.append(ms)
+    return statistics.mean(est), smp.describe(), spent
+
+
+def run_reference(args, rank, world):
+    """The reference arm: the oracle as it stands, on the host cores; each
+    step one bounded sample. Under a launcher only rank 0 works."""
+    if rank != 0:
+        return
+    cfg_name = "E" if args.config == "all" else args.config
+    smp = OracleSampler(cfg_name, args.alpha, args.gamma)
+    for _ in range(args.warmup):
+        smp.sample(rows=4)
+    walls, est = [], []
+    for _ in range(args.steps):
+        dt, ms = smp.sample(rows=4)
+        walls.append(dt)
+        est.append(ms)
+    value = statistics.mean(est)
+    cores = cpu_cores()
+    res = {"metric": METRIC, "value": round(value, 1), "unit": "ms/layer", "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup,
+           # the wall time of one sample step (the scaled per-layer estimate is `value`)
+           "ms_per_step": round(statistics.mean(walls) * 1e3, 1),
+           "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic", "impl": "reference",
+           "config": config_dict(cfg_name, args.alpha, args.gamma, world, args.shard == "heads" and world > 1),
+           "cpu_baseline": {"value": round(value, 1), "unit": "ms/layer", "cores": cores, "kind": "oracle",
+                            "sample": smp.describe() + " (one sample per step)"},
+           "e2e": {"value": round(value, 1), "unit": "ms/layer", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(res), flush=True)
 
 
 # ----------------------------------------------------------------------------- GPU arm
 
-def run_crisp(args, rank, world, local_rank):
+def load_layer(cfg_name, rank, world, heads_mode):
+    """Host tensors (q, k, v) of this rank's layer or slice, and its (h_q, h_kv)."""
     import torch
-    import torch.distributed as dist
-    import long_context_prefill_last_b200 as crisp
     from long_context_prefill_last_b200 import shard
-
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
-    c = S.CONFIGS[args.config]
+    c = S.CONFIGS[cfg_name]
     threads = min(32, os.cpu_count() or 8)
-    heads_mode = args.shard == "heads" and world > 1
     if heads_mode:
-        # one layer split by KV group: this rank draws and runs only its groups
         if world > c.h_kv:
-            raise SystemExit(f"--shard heads needs at most {c.h_kv} ranks for layer {args.config}")
+            raise SystemExit(f"--shard heads needs at most {c.h_kv} ranks for layer {cfg_name}")
         g_lo, g_hi = shard.kv_group_range(c.h_kv, world, rank)
         arrays = S.generate_slice(c, g_lo, g_hi, threads=threads)
         h_q, h_kv = (g_hi - g_lo) * c.group, g_hi - g_lo
@@ -268,59 +372,87 @@ def run_crisp(args, rank, world, local_rank):
         layer = S.generate(c, threads=threads)
         q_h, k_h, v_h = S.to_torch(layer)
         h_q, h_kv = c.h_q, c.h_kv
-    q_h, k_h, v_h = q_h.pin_memory(), k_h.pin_memory(), v_h.pin_memory()
+    return (q_h.pin_memory(), k_h.pin_memory(), v_h.pin_memory()), h_q, h_kv
+
+
+def measure(cfg_name, host, h_q, h_kv, alpha, gamma, steps, warmup, local_rank, barrier):
+    """Time K interleaved steps (CRISP step, dense reference, end-to-end) on
+    this rank; returns the per-rank measurements."""
+    import torch
+    import long_context_prefill_last_b200 as crisp
+
+    c = S.CONFIGS[cfg_name]
+    dev = torch.device("cuda", local_rank)
+    q_h, k_h, v_h = host
     q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
     out = torch.empty_like(q)
+    out_dense = torch.empty_like(q)
     out_h = torch.empty(q.shape, dtype=q.dtype).pin_memory()
     dtype = crisp.FP32 if c.dtype == "fp32" else crisp.BF16
-    cfg = crisp.Config(n=c.n, h_q=h_q, h_kv=h_kv, d=c.d, dtype=dtype, alpha=args.alpha, gamma=args.gamma)
+    cfg = crisp.Config(n=c.n, h_q=h_q, h_kv=h_kv, d=c.d, dtype=dtype, alpha=alpha, gamma=gamma)
     cfg.allocate_workspace(dev)
+    dcfg = crisp.Config(n=c.n, h_q=h_q, h_kv=h_kv, d=c.d, dtype=dtype, alpha=alpha, gamma=gamma)
+    dcfg.allocate_workspace(dev)
+    hcfg = crisp.Config(n=c.n, h_q=h_q, h_kv=h_kv, d=c.d, dtype=dtype, alpha=alpha, gamma=gamma)
+    hcfg.allocate_workspace(dev, host=True)
     ix = crisp.IndexBuffers(cfg, dev)
     stream = torch.cuda.current_stream(dev)
+    copy_stream = torch.cuda.Stream(device=dev)
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
+    def ev():
+        return torch.cuda.Event(enable_timing=True)
 
-    def step(ev_mid=None):
+    def one_step(evs=None):
+        e = evs or [None] * 7
+
+        def rec(i):
+            if e[i] is not None:
+                e[i].record(stream)
+        rec(0)
         crisp.select(q, k, cfg, ix, stream)
-        if ev_mid is not None:
-            ev_mid.record(stream)
+        rec(1)
         crisp.attend(q, k, v, out, cfg, ix, stream)
+        rec(2)
+        crisp.dense_attention(q, k, v, out_dense, dcfg, stream)
+        rec(3)
+        rec(4)
+        crisp.prefill_host(q_h, k_h, v_h, out_h, hcfg, stream, copy_stream)
+        rec(5)
 
-    # warm-up (also builds the index used for the tile count)
-    for _ in range(args.warmup):
-        step()
+    for _ in range(warmup):
+        one_step()
     crisp.raise_on_device_status(cfg, stream, "warm-up")
+    crisp.raise_on_device_status(dcfg, stream, "warm-up dense")
+    crisp.raise_on_device_status(hcfg, stream, "warm-up e2e")
     route = ix.route.cpu().numpy()
-    tiles = kept_tiles(route, ix.vs_mask.cpu().numpy().view(np.uint32), ix.pe_mask.cpu().numpy().view(np.uint32),
-                       cfg.n_blocks)
-    causal_tiles = h_q * cfg.n_blocks * (cfg.n_blocks + 1) // 2
+    tiles, pairs, union = schedule_stats(route, ix.vs_mask.cpu().numpy().view(np.uint32),
+                                         ix.pe_mask.cpu().numpy().view(np.uint32), cfg.n_blocks)
+    nb = cfg.n_blocks
 
     clocks = ClockSampler(local_rank)
     clocks.start()
-    # --- timed: the CRISP path
     barrier()
     torch.cuda.synchronize(dev)
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-            torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    for a, m, b in evs:
-        a.record(stream)
-        step(m)
-        b.record(stream)
+    evs = [[ev() for _ in range(7)] for _ in range(steps)]
+    for e in evs:
+        one_step(e)
     torch.cuda.synchronize(dev)
     barrier()
-    step_ms = [a.elapsed_time(b) for a, m, b in evs]
-    sel_ms = [a.elapsed_time(m) for a, m, b in evs]
-    att_ms = [m.elapsed_time(b) for a, m, b in evs]
     crisp.raise_on_device_status(cfg, stream, "timed steps")
+    crisp.raise_on_device_status(dcfg, stream, "timed dense")
+    crisp.raise_on_device_status(hcfg, stream, "timed e2e")
+    step_ms = [e[0].elapsed_time(e[2]) for e in evs]
+    sel_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    att_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    dense_ms = [e[2].elapsed_time(e[3]) for e in evs]
+    e2e_ms = [e[4].elapsed_time(e[5]) for e in evs]
 
-    # --- timed: the route pass alone (proxy map + finalisation + route/VS masses)
+    # the route pass alone (proxy map + finalisation + route/VS masses)
     r_out = torch.empty(h_q, dtype=torch.int32, device=dev)
     c_out = torch.empty(h_q, dtype=torch.float32, device=dev)
     crisp.route(q, k, cfg, r_out, c_out, stream)
     torch.cuda.synchronize(dev)
-    rev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    rev = [(ev(), ev()) for _ in range(steps)]
     for a, b in rev:
         a.record(stream)
         crisp.route(q, k, cfg, r_out, c_out, stream)
@@ -328,153 +460,204 @@ def run_crisp(args, rank, world, local_rank):
     torch.cuda.synchronize(dev)
     route_ms = [a.elapsed_time(b) for a, b in rev]
     crisp.raise_on_device_status(cfg, stream, "route")
-
-    # --- timed: dense reference
-    for _ in range(max(1, args.warmup // 2)):
-        crisp.dense_attention(q, k, v, out, cfg, stream)
-    barrier()
-    torch.cuda.synchronize(dev)
-    dev_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(args.dense_steps)]
-    for a, b in dev_evs:
-        a.record(stream)
-        crisp.dense_attention(q, k, v, out, cfg, stream)
-        b.record(stream)
-    torch.cuda.synchronize(dev)
-    barrier()
-    dense_ms = [a.elapsed_time(b) for a, b in dev_evs]
-    crisp.raise_on_device_status(cfg, stream, "dense")
-
-    # --- timed: end to end from page-locked host buffers through
-    # crisp_prefill_host (copies of one KV group overlap the kernels of the
-    # previous one); the device-resident copy of the layer is freed first
-    del q, k, v, out, ix
-    cfg.workspace = None
-    torch.cuda.empty_cache()
-    hcfg = crisp.Config(n=c.n, h_q=h_q, h_kv=h_kv, d=c.d, dtype=dtype, alpha=args.alpha, gamma=args.gamma)
-    hcfg.allocate_workspace(dev, host=True)
-    copy_stream = torch.cuda.Stream(device=dev)
-    crisp.prefill_host(q_h, k_h, v_h, out_h, hcfg, stream, copy_stream)   # warm-up
-    e2e_steps = max(1, min(args.steps, 3))
-    barrier()
-    torch.cuda.synchronize(dev)
-    e2e_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(e2e_steps)]
-    for a, b in e2e_evs:
-        a.record(stream)
-        crisp.prefill_host(q_h, k_h, v_h, out_h, hcfg, stream, copy_stream)
-        b.record(stream)
-    torch.cuda.synchronize(dev)
-    barrier()
-    e2e_ms = [a.elapsed_time(b) for a, b in e2e_evs]
-    crisp.raise_on_device_status(hcfg, stream, "e2e")
     clk = clocks.stop()
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    n_pe = int((route == 1).sum())
+    g_pe = len({h // (h_q // h_kv) for h in range(h_q) if route[h] == 1})
+    h2d = int(sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h)))
+    d2h = int(out_h.numel() * out_h.element_size())
+    causal_tiles = h_q * nb * (nb + 1) // 2
+    mean = statistics.mean
+    att, dense, rt = mean(att_ms), mean(dense_ms), mean(route_ms)
+    pe = max(mean(sel_ms) - rt, 1e-6)
+    rb = route_bytes(h_q, h_kv, c.n, c.d, nb)
+    sb = selection_bytes(n_pe, g_pe, c.n, c.d, nb, cfg.words)
+    # this rank's rates (per GPU)
+    rates = {"attn_tflops": 4.0 * c.d * 128 * 128 * tiles / (att * 1e-3) / 1e12,
+             "useful_tflops": 4.0 * c.d * pairs / (att * 1e-3) / 1e12,
+             "dense_tflops": 4.0 * c.d * 128 * 128 * causal_tiles / (dense * 1e-3) / 1e12,
+             "route_gbs": rb / (rt * 1e-3) / 1e9, "pe_gbs": sb / (pe * 1e-3) / 1e9,
+             "mufu_frac": (mufu_roofline(h_q * 64 * c.n, rt, clk, sms) or {}).get("frac", 0.0)}
+    return {"step_ms": step_ms, "sel_ms": sel_ms, "att_ms": att_ms, "dense_ms": dense_ms, "e2e_ms": e2e_ms,
+            "route_ms": route_ms, "tiles": tiles, "pairs": pairs, "union_tiles": union,
+            "causal_tiles": causal_tiles, "causal_pairs": h_q * c.n * (c.n + 1) // 2,
+            "heads_vs": int((route == 0).sum()), "heads_pe": n_pe, "groups_pe": g_pe,
+            "h_q": h_q, "h_kv": h_kv, "clocks": clk, "sms": sms, "h2d": h2d, "d2h": d2h,
+            "words": cfg.words, "nb": nb, "route_bytes": rb, "selection_bytes": sb, "rates": rates}
 
-    # per-rank work of this rank's launches
+
+def route_bytes(h_q, h_kv, n, d, nb):
+    """Algorithmic HBM bytes of the route pass: K read once, the proxy rows of
+    Q read once, the per-(row, tile) partials written and read back, and the
+    per-chunk statistics."""
+    rows = h_q * 64
+    return h_kv * n * d * 2 + rows * d * 2 + 2 * rows * nb * 8 + rows * ((nb + 7) // 8) * 24
+
+
+def selection_bytes(n_pe, g_pe, n, d, nb, words):
+    """Algorithmic HBM bytes of the PE pass: the PE heads' Q and their groups'
+    K read once (block pooling) and the PE masks written once."""
+    return (n_pe + g_pe) * n * d * 2 + n_pe * nb * words * 4
+
+
+RATE_KEYS = ["attn_tflops", "useful_tflops", "dense_tflops", "route_gbs", "pe_gbs", "mufu_frac"]
+
+
+def aggregate(m, world, heads_mode, dist=None, device=None):
+    """Combine the per-rank measurements: times are the maximum over ranks,
+    rates (per GPU) the minimum, i.e. the slowest rank's; with the layer split
+    by KV group, work counts add up (otherwise every rank's counts describe
+    one whole layer and are equal). Returns the combined numbers, identical
+    on every rank."""
+    import torch
+    mean = statistics.mean
+    vals = torch.tensor([mean(m["step_ms"]), mean(m["att_ms"]), mean(m["sel_ms"]), mean(m["dense_ms"]),
+                         mean(m["e2e_ms"]), mean(m["route_ms"]), statistics.median(m["step_ms"]),
+                         statistics.median(m["dense_ms"])], dtype=torch.float64, device=device)
+    rates = torch.tensor([m["rates"][k] for k in RATE_KEYS], dtype=torch.float64, device=device)
+    counts = torch.tensor([m["tiles"], m["pairs"], m["union_tiles"], m["causal_tiles"], m["causal_pairs"],
+                           m["heads_vs"], m["heads_pe"], m["groups_pe"], m["h2d"], m["d2h"]],
+                          dtype=torch.float64, device=device)
+    if world > 1 and dist is not None:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+        dist.all_reduce(rates, op=dist.ReduceOp.MIN)
+        dist.all_reduce(counts, op=dist.ReduceOp.SUM if heads_mode else dist.ReduceOp.MAX)
+    keys_v = ["step", "att", "sel", "dense", "e2e", "route", "step_median", "dense_median"]
+    keys_c = ["tiles", "pairs", "union_tiles", "causal_tiles", "causal_pairs", "heads_vs", "heads_pe",
+              "groups_pe", "h2d", "d2h"]
+    out = dict(zip(keys_v, vals.tolist()))
+    out.update(zip(RATE_KEYS, rates.tolist()))
+    out.update(zip(keys_c, (int(x) for x in counts.tolist())))
+    return out
+
+
+def result_line(cfg_name, a, m, world, heads_mode, alpha, gamma, steps, warmup):
+    """The JSON line of the CRISP arm from the aggregated numbers `a` (and
+    rank 0's own measurements `m` for the clocks)."""
+    c = S.CONFIGS[cfg_name]
     peaks, peak_src = load_peaks()
     tflops_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
     hbm_peak = peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"])
-    sms = torch.cuda.get_device_properties(dev).multi_processor_count
-    att_l, sel_l, route_l = statistics.mean(att_ms), statistics.mean(sel_ms), statistics.mean(route_ms)
-    flops = 4.0 * c.d * 128 * 128 * tiles          # computed-tile work of one attention launch
-    # algorithmic HBM bytes of the route pass: K read once, proxy rows of Q,
-    # per-(row, tile) partials written and read back, chunk statistics
-    nb = cfg.n_blocks
-    rows = h_q * 64
-    route_bytes = (h_kv * c.n * c.d * 2 + rows * c.d * 2 + 2 * rows * nb * 8
-                   + rows * ((nb + 7) // 8) * 24)
-    # selection (PE heads): their Q and their groups' K pooled once, the pooled
-    # map written once and swept by the softmax (read+write), two histogram
-    # passes and the mask pass (reads), plus the PE masks written
-    n_pe = int((route == 1).sum())
-    g_pe = len({h // c.group for h in range(h_q) if route[h] == 1})
-    tri = nb * (nb + 1) // 2
-    pe_bytes = (n_pe + g_pe) * c.n * c.d * 2 + n_pe * tri * 4 * 6 + n_pe * nb * cfg.words * 4
-    pe_ms = max(sel_l - route_l, 1e-6)
-    mufu = mufu_roofline(h_q * cfg.last_q * c.n, route_l, clk, sms)
-
-    # across ranks: times are the maximum; rates the minimum (slowest rank);
-    # with the layer split by KV group, tile and head counts add up
-    vals = torch.tensor([statistics.mean(step_ms), att_l, sel_l, statistics.mean(dense_ms),
-                         statistics.mean(e2e_ms), route_l], dtype=torch.float64, device=dev)
-    rates = torch.tensor([flops / (att_l * 1e-3) / 1e12, route_bytes / (route_l * 1e-3) / 1e9,
-                          pe_bytes / (pe_ms * 1e-3) / 1e9, (mufu or {}).get("frac", 0.0)],
-                         dtype=torch.float64, device=dev)
-    counts = torch.tensor([tiles, causal_tiles, int((route == 0).sum()), int((route == 1).sum())],
-                          dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-        dist.all_reduce(rates, op=dist.ReduceOp.MIN)
-        if heads_mode:
-            dist.all_reduce(counts, op=dist.ReduceOp.SUM)
-    step_m, att_m, sel_m, dense_m, e2e_m, route_m = vals.tolist()
-    achieved, route_gbs, pe_gbs, mufu_frac = rates.tolist()
-    tiles_all, causal_all, heads_vs, heads_pe = (int(x) for x in counts.tolist())
-    if rank != 0:
-        return None
+    clk = m["clocks"]
+    fp32 = c.dtype == "fp32"
+    achieved = a["attn_tflops"]
+    if fp32:
+        mhz = clk.get("sm_max_mhz") or 1965.0
+        peak = m["sms"] * FP32_LANES_PER_SM * 2 * mhz * 1e6 / 1e12
+        roof = {"kernel": "attn_simt_kernel (block-sparse attention, fp32 CUDA cores)", "bound": "alu",
+                "achieved": round(achieved, 3), "peak": round(peak, 1), "unit": "TFLOP/s",
+                "frac": round(achieved / peak, 4), "traffic": None,
+                "peak_source": f"derived: {m['sms']} SMs x {FP32_LANES_PER_SM} FP32 lanes x 2 flop x {mhz:g} MHz",
+                "work": "4*d*128*128 flop per computed 128x128 tile x computed tiles per launch"}
+    else:
+        src_hash = kernel_source_hash(["attn_tc.cu", "ptx.cuh"])
+        traffic = load_traffic("attn_tc_kernel", src_hash, cfg_name, alpha, gamma) if not heads_mode else None
+        roof = {"kernel": "attn_tc_kernel (block-sparse attention)", "bound": "tensor",
+                "achieved": round(achieved, 2), "peak": tflops_peak, "unit": "TFLOP/s",
+                "frac": round(achieved / tflops_peak, 4), "traffic": traffic,
+                "peak_source": f"{peak_src} bf16 dense, sustained (kernel runs inside a seconds-long step)",
+                "work": "4*d*128*128 flop per computed 128x128 tile x computed tiles per launch"}
+    mufu = mufu_roofline(m["h_q"] * 64 * c.n, a["route"], clk, m["sms"])
     if mufu is not None:
-        mufu["frac"] = round(mufu_frac, 4)
-    dense_flops = 4.0 * c.d * 128 * 128 * causal_tiles
-    h2d = int(q_h.numel() * q_h.element_size() + k_h.numel() * k_h.element_size() + v_h.numel() * v_h.element_size())
-    d2h = int(out_h.numel() * out_h.element_size())
-    src_hash = kernel_source_hash(["attn_tc.cu", "ptx.cuh"])
-    traffic = (load_traffic("attn_tc_kernel", src_hash, args.config, args.alpha, args.gamma)
-               if not heads_mode else None)
-    # whole-job ms per layer: independent layers per GPU divide by the GPUs;
-    # one layer split by KV group takes the slowest rank's time
+        mufu["frac"] = round(a["mufu_frac"], 4)
+    pe_ms = max(a["sel"] - a["route"], 1e-6)
     per_layer = 1 if heads_mode else world
     res = {
         "metric": METRIC,
-        "value": round(step_m / per_layer, 4),
+        "value": round(a["step"] / per_layer, 4),
         "unit": "ms/layer",
         "n_gpus": world,
-        "steps": args.steps,
-        "warmup": args.warmup,
-        "ms_per_step": round(step_m, 4),
+        "steps": steps,
+        "warmup": warmup,
+        "ms_per_step": round(a["step"], 4),
         "higher_is_better": False,
         "scaling": "strong" if heads_mode else "weak",
         "vs_baseline": None,
-        "dtype": "bf16" if c.dtype == "bf16" else "f32",
+        "dtype": "f32" if fp32 else "bf16",
         "data": ("synthetic (seeded Gaussian heads with planted sink/vertical/slash structure"
                  + (f", log-normal block background sigma {c.cliff_sigma:g}" if c.cliff_sigma > 0 else "")
                  + "; no datasets or weights)"),
-        "config": {"workload": f"layer {args.config}: {c.desc}", "h_q": c.h_q, "h_kv": c.h_kv, "seq_len": c.n,
-                   "alpha": args.alpha, "gamma": args.gamma,
-                   "head_dim": c.d, "batch": 1,
-                   "parallelism": (f"one layer split by KV group over {world} GPUs (no exchange)" if heads_mode
-                                   else f"independent layer per GPU x{world}"),
-                   "l2": "inputs (>= 6 GiB at 512K) far exceed the 126 MB L2; no flush between steps"},
-        "speedup_vs_dense": round(dense_m / step_m, 4),
-        "dense_ms_per_layer": round(dense_m, 4),
-        "stages_ms": {"proxy_route_select": round(sel_m, 4), "sparse_attention": round(att_m, 4)},
-        "density": {"computed_tiles": tiles_all, "causal_tiles": causal_all,
-                    "fraction": round(tiles_all / causal_all, 4), "heads_vs": heads_vs, "heads_pe": heads_pe},
+        "config": config_dict(cfg_name, alpha, gamma, world, heads_mode),
+        "speedup_vs_dense": round(a["dense"] / a["step"], 4),
+        "speedup_vs_dense_median": round(a["dense_median"] / a["step_median"], 4),
+        "dense_ms_per_layer": round(a["dense"] / per_layer, 4),
+        "timing": f"{steps} interleaved steps: CRISP step, dense attention, end-to-end call; means (medians also given)",
+        "stages_ms": {"proxy_route_select": round(a["sel"], 4), "sparse_attention": round(a["att"], 4),
+                      "crisp_step_median": round(a["step_median"], 4), "dense_median": round(a["dense_median"], 4)},
+        "density": {"computed_tiles": a["tiles"], "causal_tiles": a["causal_tiles"],
+                    "fraction": round(a["tiles"] / a["causal_tiles"], 4),
+                    "useful_pairs": a["pairs"], "causal_pairs": a["causal_pairs"],
+                    "useful_pair_fraction": round(a["pairs"] / a["causal_pairs"], 4),
+                    "cta_union_tiles": a["union_tiles"],
+                    "heads_vs": a["heads_vs"], "heads_pe": a["heads_pe"]},
+        "effective_tflops": {
+            "dense_equivalent": round(4.0 * c.d * a["causal_pairs"] / (a["step"] / per_layer * 1e-3) / 1e12, 2),
+            "useful_pairs": round(a["useful_tflops"], 2),
+            "computed_tiles": round(achieved, 2),
+            "note": "dense-equivalent = 4*d*causal pairs / CRISP step time; useful = 4*d*selected pairs / "
+                    "attention time; computed = 4*d*128*128*computed tiles / attention time"},
         "pages_speedup_context": f"{PAGES_SPEEDUP_512K}x at 512K tokens on one H100 (pages' figure, not comparable)",
-        "roofline": {"kernel": "attn_tc_kernel (block-sparse attention)", "bound": "tensor",
-                     "achieved": round(achieved, 2), "peak": tflops_peak, "unit": "TFLOP/s",
-                     "frac": round(achieved / tflops_peak, 4), "traffic": traffic,
-                     "peak_source": f"{peak_src} bf16 dense, sustained (kernel runs inside a seconds-long step)",
-                     "work": "4*d*128*128 flop per computed 128x128 tile x computed tiles per launch"},
-        "dense_tflops": round(dense_flops / (dense_m * 1e-3) / 1e12, 2),
-        "route_roofline": {"stage": "crisp_route (proxy_tc_kernel + finalize + VS masses)", "bound": "hbm",
-                           "ms": round(route_m, 4), "algorithmic_bytes": route_bytes,
-                           "achieved": round(route_gbs, 1), "peak": hbm_peak,
-                           "unit": "GB/s", "frac": round(route_gbs / hbm_peak, 4),
-                           # the proxy's exponentials (h_q x 64 x n) against MUFU at 16 per clock per SM
-                           # and the median SM clock sampled under load
+        "roofline": roof,
+        "dense_tflops": round(a["dense_tflops"], 2),
+        "route_roofline": {"stage": "crisp_route (proxy map + finalize + VS masses)", "bound": "hbm",
+                           "ms": round(a["route"], 4), "algorithmic_bytes": m["route_bytes"],
+                           "achieved": round(a["route_gbs"], 1), "peak": hbm_peak,
+                           "unit": "GB/s", "frac": round(a["route_gbs"] / hbm_peak, 4),
                            "mufu": mufu},
         "selection_roofline": {"stage": "PE pooling, pooled map, gamma cut, masks (select minus route)",
-                               "bound": "hbm", "ms": round(max(sel_m - route_m, 1e-6), 4),
-                               "algorithmic_bytes": pe_bytes,
-                               "achieved": round(pe_gbs, 1),
-                               "peak": hbm_peak, "unit": "GB/s",
-                               "frac": round(pe_gbs / hbm_peak, 4)},
-        "e2e": {"value": round(e2e_m / per_layer, 4), "unit": "ms/layer", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h,
+                               "bound": "hbm", "ms": round(pe_ms, 4), "algorithmic_bytes": m["selection_bytes"],
+                               "achieved": round(a["pe_gbs"], 1), "peak": hbm_peak, "unit": "GB/s",
+                               "frac": round(a["pe_gbs"] / hbm_peak, 4),
+                               "work": "PE heads' Q and their groups' K read once, PE masks written once"},
+        "e2e": {"value": round(a["e2e"] / per_layer, 4), "unit": "ms/layer", "h2d_bytes_per_step": a["h2d"],
+                "d2h_bytes_per_step": a["d2h"],
                 "api": "crisp_prefill_host: page-locked host buffers, copies overlapped with the kernels per KV group"},
-        "gpu_launches": KERNELS_PER_STEP * args.steps,
-        "clocks": clk,
+        # per step: crisp_select + crisp_attend, the dense launch, crisp_prefill_host (one select+attend per KV group)
+        "gpu_launches": steps * ((SELECT_KERNELS + 1) + 1 + (SELECT_KERNELS + 1) * m["h_kv"]),
+        "clocks": {k: clk.get(k) for k in ("sm_mhz", "sm_max_mhz", "reasons", "samples", "power_w_max")},
     }
     return res
+
+
+def init_dist(world):
+    if world <= 1:
+        return None
+    import datetime
+    import torch.distributed as dist
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    return dist
+
+
+def run_configs(args, rank, world, local_rank, cfg_names, settings):
+    """Measure every (config, alpha, gamma); rank 0 prints one JSON line each."""
+    import torch
+    torch.cuda.set_device(local_rank)
+    dist = init_dist(world)
+    heads_mode = args.shard == "heads" and world > 1
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    try:
+        for name in cfg_names:
+            host, h_q, h_kv = load_layer(name, rank, world, heads_mode)
+            for alpha, gamma in settings:
+                m = measure(name, host, h_q, h_kv, alpha, gamma, args.steps, args.warmup, local_rank, barrier)
+                a = aggregate(m, world, heads_mode, dist, torch.device("cuda", local_rank))
+                if rank == 0:
+                    res = result_line(name, a, m, world, heads_mode, alpha, gamma, args.steps, args.warmup)
+                    if world == 1 and not args.no_cpu_baseline and len(cfg_names) == 1 and len(settings) == 1:
+                        ms, sample, _ = oracle_ms_per_layer(name, budget_s=20.0, alpha=alpha, gamma=gamma)
+                        res["cpu_baseline"] = {"value": round(ms, 1), "unit": "ms/layer", "cores": cpu_cores(),
+                                               "kind": "oracle", "sample": sample}
+                    print(json.dumps(res), flush=True)
+                torch.cuda.empty_cache()
+            del host
+    finally:
+        if dist is not None:
+            dist.barrier()
+            dist.destroy_process_group()
 
 
 def run_stage(args):
@@ -510,20 +693,39 @@ def run_stage(args):
     torch.cuda.synchronize()
     crisp.raise_on_device_status(cfg, where=args.only)
     ms = a.elapsed_time(b) / max(1, args.steps)
-    print(json.dumps({"stage": args.only, "layer": c.name, "ms": round(ms, 4)}))
+    print(json.dumps({"stage": args.only, "layer": c.name, "n": c.n, "h_q": c.h_q, "h_kv": c.h_kv,
+                      "ms": round(ms, 4)}))
 
 
-def main():
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def launch_command(n_gpus, argv, port=None):
+    """The command that runs this script on n_gpus ranks of this node (one
+    process per GPU, rendezvous on 127.0.0.1), bounded by `timeout`."""
+    port = port or _free_port()
+    return ["timeout", "-k", "60", "3600", sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+            f"--nproc-per-node={n_gpus}", "--master-addr", "127.0.0.1", "--master-port", str(port),
+            os.path.abspath(__file__), *argv]
+
+
+def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--dense-steps", type=int, default=3)
-    ap.add_argument("--config", default="E", choices=sorted(S.CONFIGS))
+    ap.add_argument("--config", default="E", choices=sorted(S.CONFIGS) + ["all"])
     ap.add_argument("--impl", default="crisp", choices=["crisp", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--alpha", type=float, default=1.0, help="Eq. (4) noise-floor multiplier")
     ap.add_argument("--gamma", type=float, default=0.95, help="PE cumulative coverage")
+    ap.add_argument("--sweep", action="store_true",
+                    help="one line per (alpha, gamma) in {1.0, 1.25, 1.5} x {0.95, 0.97}")
     ap.add_argument("--shard", choices=["layers", "heads"], default="layers",
                     help="with N > 1 GPUs: an independent layer per GPU (weak scaling, default) or one layer "
                          "split by KV group (strong scaling)")
@@ -532,46 +734,29 @@ def main():
     ap.add_argument("--n", type=int, help="profiling mode: scaled sequence length")
     ap.add_argument("--h-q", type=int, help="profiling mode: scaled query heads")
     ap.add_argument("--h-kv", type=int, help="profiling mode: scaled KV heads")
-    args = ap.parse_args()
+    return ap.parse_args(argv)
+
+
+def main(argv=None):
+    argv = list(sys.argv[1:] if argv is None else argv)
+    args = parse_args(argv)
     if args.only:
         run_stage(args)
         return
-
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # not under a launcher: start one rank per GPU and wait for them
+        cmd = launch_command(args.gpus, argv)
+        sys.stdout.flush()
+        raise SystemExit(subprocess.call(cmd))
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-
     if args.impl == "reference":
-        if rank != 0:
-            return
-        ms, sample, spent = oracle_ms_per_layer(args.config, budget_s=max(8.0, 40.0 / max(1, args.steps)))
-        cores = cpu_cores()
-        res = {"metric": METRIC, "value": round(ms, 1), "unit": "ms/layer", "n_gpus": args.gpus,
-               "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 1), "higher_is_better": False,
-               "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-               "impl": "reference",
-               "config": {"workload": f"layer {args.config}: {S.CONFIGS[args.config].desc}"},
-               "cpu_baseline": {"value": round(ms, 1), "unit": "ms/layer", "cores": cores, "kind": "oracle",
-                                "sample": sample},
-               "e2e": {"value": round(ms, 1), "unit": "ms/layer", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
-        print(json.dumps(res))
+        run_reference(args, rank, world)
         return
-
-    if world > 1:
-        import torch.distributed as dist
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
-    res = run_crisp(args, rank, world, local_rank)
-    if rank == 0:
-        if world == 1 and not args.no_cpu_baseline:
-            ms, sample, _ = oracle_ms_per_layer(args.config, budget_s=20.0)
-            res["cpu_baseline"] = {"value": round(ms, 1), "unit": "ms/layer", "cores": cpu_cores(), "kind": "oracle",
-                                   "sample": sample}
-        print(json.dumps(res))
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
-        dist.destroy_process_group()
+    names = ALL_CONFIGS if args.config == "all" else [args.config]
+    settings = SWEEP if args.sweep else [(args.alpha, args.gamma)]
+    run_configs(args, rank, world, local_rank, names, settings)
 
 
 if __name__ == "__main__":

@@ -208,15 +208,21 @@ const char* crisp_status_string(crisp_status status);
  * - Layers needing more scratch than the array holds (about
  *   h_q * n / 128 * 640 bytes; e.g. 32 query heads up to n = 131072) are
  *   rejected with CRISP_ERR_TOO_LARGE before anything is launched.
- * - The first call on a device looks up the array's device address (once per
- *   device, with that device current); make that first call before any
- *   stream capture on the device.
+ * - The array's device address is looked up on the first call on each
+ *   device, with that device current; make that first call before any stream
+ *   capture on the device. A failed lookup is not cached (the next call tries
+ *   again). The address belongs to the device's primary context: after
+ *   cudaDeviceReset the process must not call this entry point again.
  * - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
- * - All calls share the one array and leave their contents in it: calls that
- *   can overlap on the GPU (different streams, or several host threads) race
- *   and must be serialised by the caller. Device-side conditions (a bounded
- *   wait that ran out) are recorded in the array, not in a caller workspace,
- *   so crisp_device_status does not report them. */
+ * - All calls share the one array and leave their contents in it (each call
+ *   clears what must start at zero): calls that can overlap on the GPU
+ *   (different streams, or several host threads) race and must be
+ *   serialised by the caller.
+ * - Device-side failures are reported in the outputs, since there is no
+ *   caller workspace for crisp_device_status to read: if a bounded wait ran
+ *   out or a proxy statistic was NaN or infinite (for example a NaN in the
+ *   last 64 query rows), every route[h] is -1 and every c_struct[h] NaN once
+ *   the stream completes. */
 #define CRISP_NOALLOC_SCRATCH_BYTES (32u << 20)
 crisp_status crisp_route_noalloc(const void* q, const void* k, const crisp_cfg* cfg,
                                  int32_t* route, float* c_struct, void* stream);
@@ -234,6 +240,18 @@ crisp_status crisp_exp2_selftest(const float* x, float* poly3, float* poly5, flo
  * stream completes it holds CRISP_ERR_TIMEOUT and the wait site 99. Checks
  * that a wait which runs out ends the kernel with a status, not a hang. */
 crisp_status crisp_wait_selftest(int64_t limit_cycles, int32_t* status, void* stream);
+
+/* Diagnostics: crisp_select and crisp_attend with the proxy map and the
+ * attention on the CUDA-core kernels that fp32 layers use, for bf16 layers
+ * too, so that a test can hold the tensor-core kernels against a second
+ * implementation on the same inputs. Arguments as for crisp_select and
+ * crisp_attend; dense != 0 attends over every causal key (as
+ * crisp_dense_attention; index may then be NULL). Not a production path. */
+crisp_status crisp_diag_select_simt(const void* q, const void* k, const crisp_cfg* cfg,
+                                    const crisp_index* index, void* stream);
+crisp_status crisp_diag_attend_simt(const void* q, const void* k, const void* v, void* out,
+                                    const crisp_cfg* cfg, const crisp_index* index, int32_t dense,
+                                    void* stream);
 
 /* Library version as major*10000 + minor*100 + patch. */
 int32_t crisp_version(void);

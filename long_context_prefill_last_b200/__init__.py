@@ -35,7 +35,8 @@ SYMBOLS = ["crisp_cfg_init", "crisp_workspace_size", "crisp_index_dims", "crisp_
            "crisp_attend", "crisp_prefill", "crisp_dense_attention", "crisp_device_status",
            "crisp_status_string", "crisp_version", "crisp_route_noalloc", "crisp_exp2_selftest",
            "crisp_prefill_batch", "crisp_workspace_size_batch", "crisp_prefill_varlen",
-           "crisp_prefill_host", "crisp_workspace_size_host", "crisp_wait_selftest"]
+           "crisp_prefill_host", "crisp_workspace_size_host", "crisp_wait_selftest",
+           "crisp_diag_select_simt", "crisp_diag_attend_simt"]
 
 
 def library_path() -> str:
@@ -98,6 +99,8 @@ def lib() -> ctypes.CDLL:
                                            ctypes.POINTER(vp), ctypes.POINTER(ctypes.c_int32), ctypes.c_int32,
                                            cfgp, vp]
         L.crisp_dense_attention.argtypes = [vp, vp, vp, vp, cfgp, vp]
+        L.crisp_diag_select_simt.argtypes = [vp, vp, cfgp, ctypes.POINTER(_Index), vp]
+        L.crisp_diag_attend_simt.argtypes = [vp, vp, vp, vp, cfgp, ctypes.POINTER(_Index), ctypes.c_int32, vp]
         L.crisp_device_status.argtypes = [cfgp, vp, ctypes.POINTER(ctypes.c_int32)]
         L.crisp_status_string.argtypes = [ctypes.c_int]
         L.crisp_status_string.restype = ctypes.c_char_p
@@ -244,7 +247,8 @@ def route(q, k, cfg: Config, route_out, c_struct_out, stream=None) -> None:
 def route_noalloc(q, k, cfg: Config, route_out, c_struct_out, stream=None) -> None:
     """crisp_route with the library's static scratch array instead of a workspace
     (cfg.workspace is ignored). For callers that cannot give the library device
-    memory; concurrent calls race on the shared array."""
+    memory; concurrent calls race on the shared array. A device-side failure
+    shows as route -1 and C_struct NaN on every head."""
     _check(lib().crisp_route_noalloc(_ptr(q), _ptr(k), ctypes.byref(cfg._c()), _ptr(route_out),
                                      _ptr(c_struct_out), _stream(stream)), "crisp_route_noalloc")
 
@@ -302,6 +306,20 @@ def prefill_varlen(qs, ks, vs, outs, cfg: Config, stream=None) -> None:
 def dense_attention(q, k, v, out, cfg: Config, stream=None) -> None:
     _check(lib().crisp_dense_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(out), ctypes.byref(cfg._c()),
                                        _stream(stream)), "crisp_dense_attention")
+
+
+def diag_select_simt(q, k, cfg: Config, index: IndexBuffers, stream=None) -> None:
+    """crisp_select with the proxy map on the CUDA-core kernel (a test cross-check)."""
+    _check(lib().crisp_diag_select_simt(_ptr(q), _ptr(k), ctypes.byref(cfg._c()), ctypes.byref(index._c()),
+                                        _stream(stream)), "crisp_diag_select_simt")
+
+
+def diag_attend_simt(q, k, v, out, cfg: Config, index: Optional[IndexBuffers], dense: bool = False,
+                     stream=None) -> None:
+    """crisp_attend (or dense attention) on the CUDA-core kernel (a test cross-check)."""
+    ix = ctypes.byref(index._c()) if index is not None else None
+    _check(lib().crisp_diag_attend_simt(_ptr(q), _ptr(k), _ptr(v), _ptr(out), ctypes.byref(cfg._c()), ix,
+                                        1 if dense else 0, _stream(stream)), "crisp_diag_attend_simt")
 
 
 def exp2_selftest(x, stream=None):

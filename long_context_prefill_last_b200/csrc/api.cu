@@ -56,11 +56,6 @@ WsLayout ws_layout(const Shape& s) {
   return L;
 }
 
-bool use_tensor_cores() {
-  const char* e = getenv("CRISP_FORCE_SIMT");
-  return !(e && e[0] == '1');
-}
-
 static IndexPtrs internal_index(char* ws, const WsLayout& L) {
   IndexPtrs p;
   p.route = reinterpret_cast<int32_t*>(ws + L.route);
@@ -175,11 +170,12 @@ static IndexPtrs from_abi(const crisp_index* ix) {
   } while (0)
 
 // Algorithm 2 (proxy map, finalisation, route) and Algorithm 3's selection;
-// Algorithm 4 too when `with_pe`.
+// Algorithm 4 too when `with_pe`. bf16 layers take the tensor-core proxy
+// kernel unless `simt` (the diagnostics entry points) asks for the CUDA-core one.
 static crisp_status run_index(const void* q, const void* k, const Shape& s, char* ws, const WsLayout& L,
-                              const IndexPtrs& ix, bool with_pe, cudaStream_t st) {
+                              const IndexPtrs& ix, bool with_pe, cudaStream_t st, bool simt = false) {
   CRISP_TRY(cudaMemsetAsync(ws + L.kv_pe, 0, (size_t)s.h_kv * 4, st));
-  if (!s.fp32 && use_tensor_cores())
+  if (!s.fp32 && !simt)
     CRISP_TRY(launch_proxy_tc(q, k, s, ws, L, st));
   else
     CRISP_TRY(launch_proxy_simt(q, k, s, ws, L, st));
@@ -191,9 +187,9 @@ static crisp_status run_index(const void* q, const void* k, const Shape& s, char
 
 static crisp_status run_attention(const void* q, const void* k, const void* v, void* out, const Shape& s,
                                   char* ws, const WsLayout& L, const int32_t* route, const uint32_t* vs_mask,
-                                  const uint32_t* pe_mask, bool dense, cudaStream_t st) {
+                                  const uint32_t* pe_mask, bool dense, cudaStream_t st, bool simt = false) {
   int32_t* status = reinterpret_cast<int32_t*>(ws + L.status);
-  if (!s.fp32 && use_tensor_cores())
+  if (!s.fp32 && !simt)
     CRISP_TRY(launch_attn_tc(q, k, v, out, s, route, vs_mask, pe_mask, dense, status, st));
   else
     CRISP_TRY(launch_attn_simt(q, k, v, out, s, route, vs_mask, pe_mask, dense, status, st));
@@ -511,6 +507,33 @@ crisp_status crisp_dense_attention(const void* q, const void* k, const void* v, 
   char* ws = static_cast<char*>(cfg->workspace);
   CRISP_TRY(cudaMemsetAsync(ws + L.status, 0, 32, st));
   return run_attention(q, k, v, out, s, ws, L, nullptr, nullptr, nullptr, true, st);
+}
+
+crisp_status crisp_diag_select_simt(const void* q, const void* k, const crisp_cfg* cfg, const crisp_index* index,
+                                    void* stream) {
+  Shape s;
+  WsLayout L;
+  crisp_status r = prepare(cfg, q, k, nullptr, nullptr, false, &s, &L);
+  if (r != CRISP_OK) return r;
+  if ((r = check_index(index, true)) != CRISP_OK) return r;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(cfg->workspace);
+  CRISP_TRY(cudaMemsetAsync(ws + L.status, 0, 32, st));
+  return run_index(q, k, s, ws, L, from_abi(index), true, st, true);
+}
+
+crisp_status crisp_diag_attend_simt(const void* q, const void* k, const void* v, void* out, const crisp_cfg* cfg,
+                                    const crisp_index* index, int32_t dense, void* stream) {
+  Shape s;
+  WsLayout L;
+  crisp_status r = prepare(cfg, q, k, v, out, true, &s, &L);
+  if (r != CRISP_OK) return r;
+  if (!dense && (r = check_index(index, false)) != CRISP_OK) return r;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(cfg->workspace);
+  CRISP_TRY(cudaMemsetAsync(ws + L.status, 0, 32, st));
+  if (dense) return run_attention(q, k, v, out, s, ws, L, nullptr, nullptr, nullptr, true, st, true);
+  return run_attention(q, k, v, out, s, ws, L, index->route, index->vs_mask, index->pe_mask, false, st, true);
 }
 
 crisp_status crisp_device_status(const crisp_cfg* cfg, void* stream, int32_t* device_status) {

@@ -108,7 +108,4 @@ cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, void* ou
                            const int32_t* route, const uint32_t* vs_mask, const uint32_t* pe_mask, bool dense,
                            int32_t* status, cudaStream_t st);
 
-// Whether the tensor-core (tcgen05) kernels are used for bf16 inputs.
-bool use_tensor_cores();
-
 }  // namespace crisp

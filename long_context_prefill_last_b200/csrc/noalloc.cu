@@ -4,9 +4,11 @@
 //
 // The array is a file-scope __device__ variable; host code must not pass its
 // name to a kernel (on the host the name is only a stand-in for the device
-// symbol). Its device address is looked up here once per device with
-// cudaGetSymbolAddress and that pointer is what the kernels receive.
+// symbol). Its device address is looked up here with cudaGetSymbolAddress,
+// with the device current, and that pointer is what the kernels receive.
 #include <cuda_runtime.h>
+
+#include <math.h>
 
 #include <mutex>
 
@@ -20,22 +22,42 @@ constexpr size_t kScratchBytes = CRISP_NOALLOC_SCRATCH_BYTES;
 static __device__ __align__(256) unsigned char g_route_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 64;
-std::once_flag g_once[kMaxDevices];
-void* g_scratch[kMaxDevices];
-cudaError_t g_setup[kMaxDevices];
+std::mutex g_lock[kMaxDevices];
+void* g_scratch[kMaxDevices];   // set once a lookup on that device succeeded
 
-// Device address of the array on the current device (looked up on first use).
+// Device address of the array on the current device. Only a successful
+// lookup is kept: a failed one (for example inside a stream capture) clears
+// the runtime's error and is tried again on the next call.
 cudaError_t scratch_for_device(char** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::call_once(g_once[dev], [dev] {
-    g_setup[dev] = cudaGetSymbolAddress(&g_scratch[dev], g_route_scratch);
-  });
-  if (g_setup[dev] != cudaSuccess) return g_setup[dev];
+  std::lock_guard<std::mutex> guard(g_lock[dev]);
+  if (g_scratch[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_route_scratch);
+    if (e != cudaSuccess) {
+      (void)cudaGetLastError();
+      return e;
+    }
+    g_scratch[dev] = p;
+  }
   *out = static_cast<char*>(g_scratch[dev]);
   return cudaSuccess;
+}
+
+// Copy the routes and C_struct out of the array; if any kernel of this call
+// recorded a device-side failure in the array's status word, publish
+// route = -1 and C_struct = NaN for every head instead.
+__global__ void publish_route_kernel(const int32_t* __restrict__ status, const int32_t* __restrict__ route_in,
+                                     const float* __restrict__ c_in, int32_t* __restrict__ route_out,
+                                     float* __restrict__ c_out, int h_q) {
+  const bool failed = status[0] != 0;
+  for (int h = blockIdx.x * blockDim.x + threadIdx.x; h < h_q; h += gridDim.x * blockDim.x) {
+    route_out[h] = failed ? -1 : route_in[h];
+    c_out[h] = failed ? nanf("") : c_in[h];
+  }
 }
 
 // Only the regions the route stage touches, packed from offset 0.
@@ -106,12 +128,14 @@ extern "C" crisp_status crisp_route_noalloc(const void* q, const void* k, const 
   // what must start at zero: the status word and the per-group PE flags
   if (cudaMemsetAsync(ws + L.status, 0, 32, st) != cudaSuccess) return CRISP_ERR_CUDA;
   if (cudaMemsetAsync(ws + L.kv_pe, 0, (size_t)s.h_kv * 4, st) != cudaSuccess) return CRISP_ERR_CUDA;
-  cudaError_t e = (!s.fp32 && use_tensor_cores()) ? launch_proxy_tc(q, k, s, ws, L, st)
-                                                  : launch_proxy_simt(q, k, s, ws, L, st);
+  cudaError_t e = !s.fp32 ? launch_proxy_tc(q, k, s, ws, L, st) : launch_proxy_simt(q, k, s, ws, L, st);
   if (e == cudaSuccess) e = launch_finalize(s, ws, L, ix, st);
   if (e == cudaSuccess) e = launch_vs_select(s, ws, L, ix, st);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(route, ix.route, (size_t)s.h_q * 4, cudaMemcpyDeviceToDevice, st);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(c_struct, ix.c_struct, (size_t)s.h_q * 4, cudaMemcpyDeviceToDevice, st);
+  if (e == cudaSuccess) {
+    publish_route_kernel<<<(s.h_q + 255) / 256, 256, 0, st>>>(reinterpret_cast<const int32_t*>(ws + L.status),
+                                                              ix.route, ix.c_struct, route, c_struct, s.h_q);
+    e = cudaGetLastError();
+  }
   if (e != cudaSuccess) {
     (void)cudaGetLastError();
     return CRISP_ERR_CUDA;

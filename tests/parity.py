@@ -6,8 +6,13 @@
   relative of alpha*mu (a flip).
 * PE masks: bit-exact, except an entry whose oracle value lies within 1e-3
   relative of the oracle's cut value (a flip).
-* Outputs on the same indices: max |o - o_ref| / max |o_ref| per head within
-  2e-2 (bf16) or 1e-4 (fp32).
+* Outputs on the same indices: two normalisations of the max error, each
+  within 2e-2 (bf16) or 1e-4 (fp32):
+  - per head: max |o - o_ref| / max |o_ref| over the head's checked rows;
+  - per row: max over rows of max_c |o - o_ref| / max_c |o_ref| (a row with a
+    small output is measured against its own size, not the head's largest).
+* Flip counts are reported per head and kind, and bounded: at most 1% of a
+  head's VS blocks (2 N_b) or of its causal PE blocks.
 """
 from __future__ import annotations
 
@@ -17,6 +22,7 @@ from typing import Dict, List
 import numpy as np
 
 REL_FLIP = 1e-3
+FLIP_FRAC_MAX = 0.01
 TOL = {"bf16": 2e-2, "fp32": 1e-4}
 
 
@@ -51,6 +57,21 @@ class Report:
 
     def assert_ok(self):
         assert not self.failures, "\n".join(self.failures[:20])
+
+    def summary(self) -> str:
+        vs = sum(self.vs_flips.values())
+        pe = sum(self.pe_flips.values())
+        worst_vs = max(self.vs_flips.items(), key=lambda kv: kv[1], default=(None, 0))
+        worst_pe = max(self.pe_flips.items(), key=lambda kv: kv[1], default=(None, 0))
+        return (f"flips: route {len(self.route_flips)} heads {self.route_flips}; VS blocks {vs} "
+                f"(max {worst_vs[1]} on head {worst_vs[0]}); PE blocks {pe} (max {worst_pe[1]} on head {worst_pe[0]})")
+
+    def assert_flips_bounded(self, nb: int, frac: float = FLIP_FRAC_MAX):
+        """Each head's flips stay a small fraction of its candidates."""
+        for h, c in self.vs_flips.items():
+            assert c <= frac * 2 * nb, f"head {h}: {c} VS flips of {2 * nb} blocks"
+        for h, c in self.pe_flips.items():
+            assert c <= frac * nb * (nb + 1) / 2, f"head {h}: {c} PE flips of {nb * (nb + 1) // 2} blocks"
 
 
 def compare_route(h, c_gpu, route_gpu, idx, tau, rep: Report):
@@ -100,4 +121,12 @@ def compare_pe(h, mask_gpu, idx, rep: Report):
 
 
 def output_error(o_gpu: np.ndarray, o_ref: np.ndarray) -> float:
+    """max |o - o_ref| / max |o_ref| over the whole array (one head's rows)."""
     return float(np.max(np.abs(o_gpu - o_ref)) / max(np.max(np.abs(o_ref)), 1e-30))
+
+
+def row_error(o_gpu: np.ndarray, o_ref: np.ndarray) -> float:
+    """max over rows of max_c |o - o_ref| / max_c |o_ref| (rows: [rows, d])."""
+    num = np.max(np.abs(o_gpu - o_ref), axis=-1)
+    den = np.maximum(np.max(np.abs(o_ref), axis=-1), 1e-30)
+    return float(np.max(num / den))

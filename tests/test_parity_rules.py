@@ -45,3 +45,27 @@ def test_vs_mismatch_far_from_threshold_fails_near_is_flip():
     rep = P.Report()
     P.compare_vs(0, gpu2, idx.sel_s, idx, 1.0, rep)
     assert not rep.failures and rep.vs_flips[0] == 1
+
+
+def test_row_error_measures_each_row_against_its_own_size():
+    ref = np.array([[10.0, -10.0, 1.0], [0.01, 0.02, -0.01]])
+    gpu = ref.copy()
+    gpu[1, 1] += 0.001                 # 0.001 off a row whose largest entry is 0.02
+    assert abs(P.output_error(gpu, ref) - 0.001 / 10.0) < 1e-12
+    assert abs(P.row_error(gpu, ref) - 0.001 / 0.02) < 1e-12
+    assert P.row_error(ref, ref) == 0.0
+
+
+def test_flip_bound_is_per_head_and_per_kind():
+    rep = P.Report()
+    rep.vs_flips = {0: 1, 1: 0}
+    rep.pe_flips = {2: 3}
+    rep.assert_flips_bounded(nb=64)    # 1 of 128 VS blocks, 3 of 2080 PE blocks
+    assert "VS blocks 1" in rep.summary() and "PE blocks 3" in rep.summary()
+    rep.vs_flips[1] = 2                # 2 of 128 VS blocks: above 1%
+    try:
+        rep.assert_flips_bounded(nb=64)
+    except AssertionError:
+        pass
+    else:
+        raise AssertionError("2 of 128 VS flips exceeds 1%")

@@ -6,8 +6,12 @@ Its scratch is a static device array inside the library, shared by every
 call, so two calls in a row must not see each other's leftovers: each call
 is compared with crisp_route (which uses a caller workspace) on a different
 layer, with the tolerance the parity tests use for C_struct and exact routes.
-This file is collected last so that, if it fails, a run that stops at the
-first failure has already run every other test.
+A device-side failure cannot be read from a caller workspace here (there is
+none), so the entry point reports it in its outputs: a NaN in a proxy row
+must come back as route -1 and C_struct NaN on every head, and the next call
+on good inputs must be normal again. This file is collected last so that, if
+it fails, a run that stops at the first failure has already run every other
+test.
 """
 import numpy as np
 import pytest
@@ -50,3 +54,21 @@ def test_route_noalloc_matches_route_on_two_calls_in_a_row():
         assert (r_na == r_ref).all(), (lc.name, r_na, r_ref)
         np.testing.assert_allclose(c_na, c_ref, rtol=1e-4, atol=1e-4)
         assert set(np.unique(r_na)) <= {0, 1}
+
+
+def test_route_noalloc_reports_a_device_failure_in_its_outputs():
+    from long_context_prefill_last_b200 import build
+    build.build()
+    layer = S.generate(S.scaled("B", n=4096, h_q=8, h_kv=2), with_v=False)
+    q, k, _ = (t.cuda() for t in S.to_torch(layer))
+    cfg = crisp.Config(n=4096, h_q=8, h_kv=2)
+    bad = q.clone()
+    bad[3, -5, :] = float("nan")                 # one of the 64 proxy rows of query head 3
+    r = torch.zeros(8, dtype=torch.int32, device="cuda")
+    c = torch.zeros(8, dtype=torch.float32, device="cuda")
+    crisp.route_noalloc(bad, k, cfg, r, c)
+    torch.cuda.synchronize()
+    assert (r.cpu() == -1).all() and torch.isnan(c.cpu()).all()
+    crisp.route_noalloc(q, k, cfg, r, c)         # the next call starts clean
+    torch.cuda.synchronize()
+    assert set(r.cpu().tolist()) <= {0, 1} and torch.isfinite(c.cpu()).all()
