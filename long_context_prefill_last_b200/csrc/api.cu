@@ -31,13 +31,16 @@ WsLayout ws_layout(const Shape& s) {
   L.chunk_w = take(rows * s.n_chunks * 4);
   L.tile_a = take(hq * nb * 4);
   L.tile_b = take(hq * nb * 4);
-  L.qbar = take(hq * nb * kHeadDim * 4);
-  L.kbar = take(hkv * nb * kHeadDim * 4);
-  L.tri = take(hq * (size_t)s.tri_stride * 4);
-  L.tri_stats = take(hq * nb * (size_t)((s.nb + 63) / 64) * 16);
+  const size_t nb_pad = (size_t)s.nt * 128;
+  L.qhi = take(hq * nb * kHeadDim * 2);
+  L.qlo = take(hq * nb * kHeadDim * 2);
+  L.khi = take(hkv * nb_pad * kHeadDim * 2);
+  L.klo = take(hkv * nb_pad * kHeadDim * 2);
+  L.row_stat = take(hq * nb * 8);
+  L.tile_kr = take(hq * (size_t)s.nt * s.nt * 4 * 8);
+  L.tie_cnt = take(hq * nb * (size_t)s.nt * 4);
   L.hist = take(hq * sizeof(PeHist));
   L.pe_state = take(hq * sizeof(PeState));
-  L.tie_rows = take(hq * nb * 4);
   L.kv_pe = take(hkv * 4);
   L.route = take(hq * 4);
   L.c_struct = take(hq * 4);
@@ -97,8 +100,7 @@ static crisp_status make_shape(const crisp_cfg* c, Shape* s) {
   s->words = (s->nb + 31) / 32;
   s->n_chunks = (s->nb + kChunkTiles - 1) / kChunkTiles;
   s->last_q = c->last_q;
-  s->tri = (long long)s->nb * (s->nb + 1) / 2;
-  s->tri_stride = (s->tri + 63) & ~63LL;
+  s->nt = (s->nb + 127) / 128;
   s->fp32 = c->dtype == CRISP_FP32;
   s->sm_scale = c->sm_scale > 0.f ? c->sm_scale : 1.f / sqrtf((float)c->d);
   s->scale_log2 = s->sm_scale * 1.4426950408889634f;

@@ -26,13 +26,13 @@ struct WsLayout {
   size_t chunk_w;     // f32 [h_q][last_q][n_chunks] weight of each chunk's partials
   size_t tile_a;      // f32 [h_q][N_b]  sum over rows of weighted part_lo
   size_t tile_b;      // f32 [h_q][N_b]  sum over rows of weighted part_hi
-  size_t qbar;        // f32 [h_q][N_b][d]
-  size_t kbar;        // f32 [h_kv][N_b][d]
-  size_t tri;         // f32 [h_q][N_b(N_b+1)/2]  normalised pooled map, row-major triangle
-  size_t tri_stats;   // f32x4 [h_q][N_b][ceil(N_b/64)] (max, sum of 2^(l - max), min, 0) of each row's 64-column tiles
+  size_t qhi, qlo;    // bf16 [h_q][N_b][d]          pooled Q * scale_log2, hi and lo parts
+  size_t khi, klo;    // bf16 [h_kv][nt*128][d]      pooled K, hi and lo parts (rows past N_b zero)
+  size_t row_stat;    // f32x2 [h_q][N_b]            pooled-map row (maximum, 1 / (sum * N_b)), log2 domain
+  size_t tile_kr;     // u32x2 [h_q][nt][nt][4]      (min, max) key of each 32-row quarter of a 128x128 map tile
+  size_t tie_cnt;     // u32 [h_q][N_b][nt]          entries equal to the cut per (row, tile), then offsets
   size_t hist;        // per head: PeHist
   size_t pe_state;    // per head: PeState
-  size_t tie_rows;    // u32 [h_q][N_b] ties per row, then exclusive offsets
   size_t kv_pe;       // int32 [h_kv]: 1 if any query head of the group routes PE
   // internal index (used by crisp_prefill / crisp_route)
   size_t route, c_struct, p_v, p_s, mu, vs_mask, v_idx, s_idx, nv, ns, pe_mask, pe_count, pe_cut;
@@ -41,8 +41,7 @@ struct WsLayout {
 
 struct Shape {
   int n, h_q, h_kv, d, group, nb, words, n_chunks, last_q;
-  long long tri;         // entries of the causal block triangle
-  long long tri_stride;  // floats reserved per head for it (tri rounded up to 64)
+  int nt;                // 128-block tiles of the pooled map per side: ceil(N_b / 128)
   bool fp32;
   float sm_scale;     // natural-log domain scale
   float scale_log2;   // sm_scale * log2(e)

@@ -1,65 +1,77 @@
-// Pooled estimation (CRISP summary page, Algorithm 4, "GlobalAdaptive"):
-// block-mean pooling of Q and K, A-bar = softmax(Q-bar K-bar^T * sm_scale)
-// over c <= r, normalisation of the flattened causal map by its total (N_b,
-// one per row), and the gamma-cumulative cut: keep the largest entries
-// (ties by ascending flat index r*N_b + c) until their mass reaches gamma.
-// The diagonal block is always kept.
+// Pooled estimation (CRISP summary page, Algorithm 4, "GlobalAdaptive") on
+// the 5th-generation tensor cores.
 //
-// The cut is found without sorting: a three-level radix select over the
-// fp32 bit patterns of the (positive) entries, with per-bucket counts and
-// float64 mass. Only heads routed PE do any work; the rest exit at once.
+// What is computed, per query head routed PE: block means Q-bar, K-bar of Q
+// and K (B = 128 rows), the pooled map A-bar = softmax over c <= r of
+// sm_scale * Q-bar_r . K-bar_c, its flattened causal entries divided by their
+// total (N_b, one per row), and the gamma-cumulative cut: the largest entries
+// (ties by ascending flat index r*N_b + c) are kept until their mass reaches
+// gamma. The diagonal block is always kept.
+//
+// How: the cut is found by a three-level radix select over the fp32 bit
+// patterns of the (positive) entries, with per-bucket counts and float64
+// mass, and the map is never stored. Every pass recomputes the pooled
+// logits it needs on the tensor cores: Q-bar * scale and K-bar are split into
+// bf16 hi + lo parts and S = Qh.Kh^T + Ql.Kh^T + Qh.Kl^T (the lo.lo term is
+// below fp32 rounding), with Q-bar held in tensor memory as the A operand
+// and K-bar tiles fed by TMA. The passes:
+//   1. stats + level-0: per 128-row stripe of the map, one sweep computes
+//      each row's maximum and normaliser (online softmax), a second sweep
+//      the entries, their level-0 histogram (bits 31..20) and, per tile, the
+//      smallest and largest key;
+//   2. level 1 (bits 19..8) and level 2 (bits 7..0): only tiles whose key
+//      range meets the prefix found so far are recomputed;
+//   3. ties (only when the cut keeps part of the entries equal to it): per
+//      (row, tile) counts of entries equal to the cut, then a scan in flat
+//      order;
+//   4. masks: tiles entirely above (below) the cut are written without
+//      recomputation; the rest are recomputed and compared.
+#include <cuda.h>
 #include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
 
 #include "internal.h"
 #include "ptx.cuh"
+#include "tmap.h"
 
 namespace crisp {
 namespace {
 
+enum PeMode : int { kStatsHist0 = 0, kHist1 = 1, kHist2 = 2, kTies = 3, kMask = 4 };
+
 struct PeArgs {
-  int n, nb, words, group, h_q, h_kv;
-  long long tri, tri_stride;
-  float scale_log2;
+  int nb, nt, words, group, h_q;
   float gamma;
   const int32_t* route;
-  const int32_t* kv_pe;
-  float* qbar;
-  float* kbar;
-  float* tri_buf;
-  float4* tri_stats;   // [h_q][nb][n_ct] per-tile row (max, sum of 2^(l - max), min, 0)
-  int n_ct;            // 64-column tiles per row
+  const __nv_bfloat16* qhi;   // [h_q][nb][128]  bf16(Q-bar * scale_log2)
+  const __nv_bfloat16* qlo;   // [h_q][nb][128]  bf16(Q-bar * scale_log2 - qhi)
+  float2* row_stat;           // [h_q][nb]        (row maximum, 1 / (row sum * N_b)), log2 domain
+  uint2* tile_kr;             // [h_q][nt][nt][4] (min key, max key) per 32-row quarter of a tile
+  uint32_t* tie_cnt;          // [h_q][nb][nt]    ties per (row, tile), then exclusive offsets
   PeHist* hist;
   PeState* state;
-  uint32_t* tie_rows;
   uint32_t* pe_mask;
   int64_t* pe_count;
   float* pe_cut;
   int32_t* status;
 };
 
-__device__ __forceinline__ long long tri_off(int r) { return (long long)r * (r + 1) / 2; }
+// ------------------------------------------------------------------ pooling
 
-__device__ __forceinline__ float warp_max(float v) {
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
-}
-__device__ __forceinline__ float warp_min(float v) {
-  for (int o = 16; o > 0; o >>= 1) v = fminf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
-}
-__device__ __forceinline__ float warp_sum(float v) {
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
-
-// 16 bytes of T widened to fp32.
+// Block means of Q (query heads routed PE) and K (KV groups with a PE head),
+// written as bf16 hi/lo pairs; Q-bar is scaled by sm_scale * log2(e) first so
+// the logits come out in the log2 domain. Persistent grid over (head, block)
+// items; one 128 x 128 block per CTA iteration, every load issued before the
+// first add (32 KB in flight per CTA).
 template <typename T>
 struct Vec16;
 template <>
 struct Vec16<__nv_bfloat16> {
   static constexpr int N = 8;
   __device__ static void load(const __nv_bfloat16* p, float (&o)[8]) {
-    const uint4 u = *reinterpret_cast<const uint4*>(p);
+    const uint4 u = __ldcs(reinterpret_cast<const uint4*>(p));
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -72,7 +84,7 @@ template <>
 struct Vec16<float> {
   static constexpr int N = 4;
   __device__ static void load(const float* p, float (&o)[4]) {
-    const float4 u = *reinterpret_cast<const float4*>(p);
+    const float4 u = __ldcs(reinterpret_cast<const float4*>(p));
     o[0] = u.x;
     o[1] = u.y;
     o[2] = u.z;
@@ -80,292 +92,660 @@ struct Vec16<float> {
   }
 };
 
-// Block mean of 128 rows of x[head] -> out[head][b][:] (fp32). One CTA per
-// (block, head); 16-byte loads, 128 / N threads per row, N rows at a time.
+constexpr int kPoolThreads = 256;
+
 template <typename T>
-__global__ void __launch_bounds__(128) pool_kernel(const T* __restrict__ x, float* __restrict__ out, int n, int nb,
-                                                   const int32_t* __restrict__ flag) {
-  const int b = blockIdx.x, head = blockIdx.y;
-  if (flag[head] == 0) return;   // route (query heads) or PE-group flag (KV heads)
+__global__ void __launch_bounds__(kPoolThreads) pe_pool_kernel(const T* __restrict__ q, const T* __restrict__ k,
+                                                               int n, int nb, int nb_pad, int h_q, int h_kv,
+                                                               float scale, const int32_t* __restrict__ route,
+                                                               const int32_t* __restrict__ kv_pe,
+                                                               __nv_bfloat16* __restrict__ qhi,
+                                                               __nv_bfloat16* __restrict__ qlo,
+                                                               __nv_bfloat16* __restrict__ khi,
+                                                               __nv_bfloat16* __restrict__ klo) {
   constexpr int N = Vec16<T>::N;
-  constexpr int TPR = kHeadDim / N;   // threads per row
-  constexpr int RP = 128 / TPR;       // rows in parallel
-  __shared__ float red[RP][kHeadDim];
+  constexpr int TPR = kHeadDim / N;            // threads per row
+  constexpr int RP = kPoolThreads / TPR;       // rows in parallel
+  constexpr int IT = kBlock / RP;              // rows per thread
+  __shared__ float red[RP][kHeadDim + 1];
   const int tid = threadIdx.x, rg = tid / TPR, c0 = (tid % TPR) * N;
-  float acc[N];
+  // items: query heads x N_b blocks, then KV heads x nb_pad blocks (K-bar rows
+  // past N_b are written as zeros so its TMA boxes never leave the tensor)
+  const long long q_items = (long long)h_q * nb;
+  const long long items = q_items + (long long)h_kv * nb_pad;
+  for (long long it = blockIdx.x; it < items; it += gridDim.x) {
+    const bool is_q = it < q_items;
+    const int hh = is_q ? (int)(it / nb) : (int)((it - q_items) / nb_pad);
+    const int b = is_q ? (int)(it % nb) : (int)((it - q_items) % nb_pad);
+    const bool want = is_q ? route[hh] == 1 : kv_pe[hh] != 0;
+    if (!want) continue;   // uniform over the CTA
+    float acc[N];
 #pragma unroll
-  for (int j = 0; j < N; ++j) acc[j] = 0.f;
-  const T* base = x + ((size_t)head * n + (size_t)b * kBlock) * kHeadDim + c0;
-#pragma unroll 4
-  for (int row = rg; row < kBlock; row += RP) {
-    float v[N];
-    Vec16<T>::load(base + (size_t)row * kHeadDim, v);
+    for (int j = 0; j < N; ++j) acc[j] = 0.f;
+    if (b < nb) {
+      const T* base = (is_q ? q : k) + ((size_t)hh * n + (size_t)b * kBlock) * kHeadDim + c0;
+      float v[IT][N];
 #pragma unroll
-    for (int j = 0; j < N; ++j) acc[j] += v[j];
+      for (int i = 0; i < IT; ++i) Vec16<T>::load(base + (size_t)(rg + i * RP) * kHeadDim, v[i]);
+#pragma unroll
+      for (int j = 0; j < N; ++j) {
+        float s = 0.f;
+#pragma unroll
+        for (int i = 0; i < IT; ++i) s += v[i][j];
+        acc[j] = s;
+      }
+    }
+    __syncthreads();   // the previous item's reads of red are done
+#pragma unroll
+    for (int j = 0; j < N; ++j) red[rg][c0 + j] = acc[j];
+    __syncthreads();
+    if (tid < kHeadDim) {
+      float s = 0.f;
+#pragma unroll
+      for (int g = 0; g < RP; ++g) s += red[g][tid];
+      const float x = s * (1.f / kBlock) * (is_q ? scale : 1.f);
+      const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+      const __nv_bfloat16 lo = __float2bfloat16_rn(x - __bfloat162float(hi));
+      const size_t o = ((size_t)hh * (is_q ? nb : nb_pad) + b) * kHeadDim + tid;
+      (is_q ? qhi : khi)[o] = hi;
+      (is_q ? qlo : klo)[o] = lo;
+    }
   }
-#pragma unroll
-  for (int j = 0; j < N; ++j) red[rg][c0 + j] = acc[j];
-  __syncthreads();
-  float s = 0.f;
-#pragma unroll
-  for (int g = 0; g < RP; ++g) s += red[g][tid];
-  out[((size_t)head * nb + b) * kHeadDim + tid] = s * (1.f / kBlock);
 }
 
-// Pooled logits (log2 domain) of one 128 x 128 tile (rt, ct), ct <= rt, of
-// the block-causal triangle. Thread (ty, tx) holds an 8 x 8 register tile:
-// rows ty*4 + {0..3} and 64 + ty*4 + {0..3}, columns tx*4 + {0..3} and
-// 64 + tx*4 + {0..3}. Both operand tiles sit transposed in shared memory
-// ([d][block], row stride 132 floats), so each step over d reads four float4
-// (contiguous across the threads of a row) for 64 FMAs. The statistics the
-// row softmax needs are kept per 64-column half (kLT).
-constexpr int kLT = 64;        // columns per statistics tile
-constexpr int kLT2 = 128;      // blocks per CTA tile side
-constexpr int kLStride = 132;  // floats per transposed row
-// One tile ti of query head h (routed PE).
-__device__ __forceinline__ void pe_logits_tile(const PeArgs& a, int h, int ti, float* lsm) {
-  const int g = h / a.group;
-  // linear lower-triangle tile index -> (rt, ct)
-  int rt = (int)((sqrtf(8.f * (float)ti + 1.f) - 1.f) * 0.5f);
-  while ((rt + 1) * (rt + 2) / 2 <= ti) ++rt;
-  while (rt * (rt + 1) / 2 > ti) --rt;
-  const int ct = ti - rt * (rt + 1) / 2;
-  const int r0 = rt * kLT2, c0 = ct * kLT2;
-  float* qT = lsm;                        // [128][kLStride]
-  float* kT = lsm + kHeadDim * kLStride;  // [128][kLStride]
-  const int tid = threadIdx.x;
-  for (int e = tid; e < kLT2 * kHeadDim; e += 256) {
-    const int rr = e >> 7, dd = e & 127;
-    qT[dd * kLStride + rr] =
-        (r0 + rr < a.nb) ? a.qbar[((size_t)h * a.nb + r0 + rr) * kHeadDim + dd] * a.scale_log2 : 0.f;
-    kT[dd * kLStride + rr] = (c0 + rr < a.nb) ? a.kbar[((size_t)g * a.nb + c0 + rr) * kHeadDim + dd] : 0.f;
+// ------------------------------------------------------------------ the tensor-core sweep
+
+// warp 0 TMA, warp 1 TMEM + MMA, warps 2-3 idle, warps 4..11 two epilogue
+// warpgroups; the first warpgroup gives registers to the epilogue ones
+// (setmaxnreg 64 / 216 / 216; 128*64 + 256*216 <= 384*168, the launch allocation)
+constexpr int kThreads = 384;
+constexpr int kRegsControl = 64;
+constexpr int kRegsEpilogue = 216;
+static_assert(128 * kRegsControl + 256 * kRegsEpilogue <= kThreads * 168, "register split exceeds the launch");
+constexpr int kStages = 2;
+constexpr uint32_t kTileBytes = 128 * 128 * 2;   // one bf16 128 x 128 tile (two 64-column halves)
+constexpr uint32_t kHalfBytes = 128 * 128;
+constexpr int kHistMax = kHistL1;                // largest per-CTA histogram (level 1)
+constexpr uint32_t OFF_K = 0;                                      // [stage][hi, lo] K-bar tiles
+constexpr uint32_t OFF_HCNT = OFF_K + kStages * 2 * kTileBytes;    // u32 [kHistMax]
+constexpr uint32_t OFF_HMASS = OFF_HCNT + kHistMax * 4;            // f64 [kHistMax]
+constexpr uint32_t OFF_XCH = OFF_HMASS + kHistMax * 8;             // float2 [128]: row statistics exchange
+constexpr uint32_t OFF_ROW = OFF_XCH + 128 * 8;                    // float2 [128]: (m, inv) of the stripe's rows
+constexpr uint32_t OFF_BAR = OFF_ROW + 128 * 8;
+enum {
+  B_KFULL = 0,
+  B_KEMPTY = B_KFULL + kStages,
+  B_SFULL = B_KEMPTY + kStages,   // [2]
+  B_SEMPTY = B_SFULL + 2,         // [2], 128 arrivals (one warpgroup)
+  B_QFULL = B_SEMPTY + 2,         // [2], 256 arrivals (both warpgroups)
+  B_QEMPTY = B_QFULL + 2,         // [2], MMA commit after a stripe's last tile
+  B_EPI = B_QEMPTY + 2,           // epilogue-wide sync, 256 arrivals
+  B_DRAIN = B_EPI + 1,
+  B_COUNT = B_DRAIN + 1
+};
+constexpr uint32_t OFF_ABORT = OFF_BAR + 8 * B_COUNT;
+constexpr uint32_t OFF_TMEMPTR = OFF_ABORT + 4;
+constexpr uint32_t kSmemBytes = OFF_TMEMPTR + 4 + 1024;
+static_assert(kSmemBytes <= 232448, "shared memory budget");
+// TMEM: S[0] cols [0,128), S[1] [128,256); Q[b] at 256 + 128 b: hi [0,64), lo [64,128)
+constexpr uint32_t kTmemCols = 512;
+
+__device__ __forceinline__ uint32_t bar_addr(uint32_t base, int i) { return base + OFF_BAR + 8u * i; }
+
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag, int32_t* status,
+                                          int where) {
+  const bool ok = dev::mbar_wait(bar, parity, abort_flag, status, where);
+  return __all_sync(0xffffffffu, ok);
+}
+
+__device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile_base, int kk) {
+  return dev::smem_desc_sw128(tile_base + (kk >> 2) * kHalfBytes + (kk & 3) * 32, 16, 1024);
+}
+
+// The value of one map entry from its log2-domain logit and its row's (m, inv);
+// every pass evaluates exactly this expression, so they all see the same bits.
+__device__ __forceinline__ float entry_value(float l, float m, float inv) { return dev::ex2(l - m) * inv; }
+
+// Item i of CTA b (snake over items ordered longest stripe first): (head, row tile) or false.
+__device__ __forceinline__ bool item_of(const PeArgs& a, int b, int k, int& h, int& rt) {
+  const int G = gridDim.x;
+  const long long idx = (k & 1) ? (long long)(k + 1) * G - 1 - b : (long long)k * G + b;
+  if (idx >= (long long)a.h_q * a.nt) return false;
+  rt = a.nt - 1 - (int)(idx / a.h_q);
+  h = (int)(idx % a.h_q);
+  return true;
+}
+
+struct PassCtx {
+  int mode;
+  uint32_t lo_key, hi_key;   // keys a tile must reach to be recomputed
+  uint32_t cut;              // level-2 result (ties, mask)
+  bool all;                  // the cut keeps every entry
+  bool partial_ties;
+  unsigned long long t_keep;
+  uint32_t prefix;
+};
+
+// Whether head h takes part in this pass, and its pass parameters.
+__device__ __forceinline__ bool head_live(const PeArgs& a, int mode, int h, PassCtx& c) {
+  if (a.route[h] != 1) return false;
+  c.mode = mode;
+  if (mode == kStatsHist0) return true;
+  const PeState* st = a.state + h;
+  c.all = st->all != 0;
+  c.cut = st->cut_key;
+  c.prefix = st->prefix;
+  c.t_keep = st->t_keep;
+  c.partial_ties = !c.all && st->t_keep < st->n_ties;
+  if (mode == kHist1) {
+    c.lo_key = c.prefix << 20;
+    c.hi_key = c.lo_key | 0xFFFFFu;
+    return !c.all;
+  }
+  if (mode == kHist2) {
+    c.lo_key = c.prefix << 8;
+    c.hi_key = c.lo_key | 0xFFu;
+    return !c.all;
+  }
+  c.lo_key = c.hi_key = c.cut;
+  if (mode == kTies) return c.partial_ties;
+  return true;   // kMask
+}
+
+// Key range of tile (rt, ct) of head h recorded by the level-0 sweep.
+__device__ __forceinline__ void tile_range(const PeArgs& a, int h, int rt, int ct, uint32_t& kmin, uint32_t& kmax) {
+  const uint2* p = a.tile_kr + (((size_t)h * a.nt + rt) * a.nt + ct) * 4;
+  kmin = 0xFFFFFFFFu;
+  kmax = 0u;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint2 e = p[q];
+    kmin = min(kmin, e.x);
+    kmax = max(kmax, e.y);
+  }
+}
+
+// Whether tile (rt, ct) is recomputed on the tensor cores in this pass.
+__device__ __forceinline__ bool tile_active(const PeArgs& a, const PassCtx& c, int h, int rt, int ct) {
+  if (c.mode == kStatsHist0) return true;
+  if (c.mode == kMask && c.all) return false;
+  uint32_t kmin, kmax;
+  tile_range(a, h, rt, ct, kmin, kmax);
+  return kmin <= c.hi_key && kmax >= c.lo_key;
+}
+
+// The tiles ct <= rt of stripe (h, rt) recomputed in this pass, as a bit mask
+// (N_b <= 8192, so at most 64 tiles). Evaluated by a whole warp, one tile per
+// lane, so the key ranges are read in one round.
+__device__ __forceinline__ uint64_t stripe_mask(const PeArgs& a, const PassCtx& c, int h, int rt, int lane) {
+  const bool a0 = lane <= rt && tile_active(a, c, h, rt, lane);
+  const bool a1 = lane + 32 <= rt && tile_active(a, c, h, rt, lane + 32);
+  return (uint64_t)__ballot_sync(0xffffffffu, a0) | ((uint64_t)__ballot_sync(0xffffffffu, a1) << 32);
+}
+
+// The tiles ct <= rt of stripe (h, rt) whose every entry lies above the cut
+// (kept whole by the mask pass without recomputation); warp-wide like stripe_mask.
+__device__ __forceinline__ uint64_t stripe_above(const PeArgs& a, const PassCtx& c, int h, int rt, int lane) {
+  uint32_t kmin, kmax;
+  bool a0 = false, a1 = false;
+  if (lane <= rt) {
+    tile_range(a, h, rt, lane, kmin, kmax);
+    a0 = kmin > c.cut;
+  }
+  if (lane + 32 <= rt) {
+    tile_range(a, h, rt, lane + 32, kmin, kmax);
+    a1 = kmin > c.cut;
+  }
+  return (uint64_t)__ballot_sync(0xffffffffu, a0) | ((uint64_t)__ballot_sync(0xffffffffu, a1) << 32);
+}
+
+__device__ __forceinline__ int sweeps_of(int mode) { return mode == kStatsHist0 ? 2 : 1; }
+
+// Epilogue-wide barrier (256 threads) with a bounded wait.
+__device__ __forceinline__ bool epi_sync(uint32_t sbase, uint32_t& phase, volatile int* abort_flag,
+                                         int32_t* status) {
+  dev::mbar_arrive(bar_addr(sbase, B_EPI));
+  const bool ok = warp_wait(bar_addr(sbase, B_EPI), phase, abort_flag, status, 40);
+  phase ^= 1u;
+  return ok;
+}
+
+__device__ __forceinline__ void hist_add(uint32_t* cnt, double* mass, uint32_t b, uint32_t c, double m) {
+  atomicAdd(&cnt[b], c);
+  atomicAdd(&mass[b], m);
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kThreads, 1)
+pe_sweep_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constant__ CUtensorMap tm_klo, PeArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t raw = dev::smem_u32(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  uint8_t* sgen = smem_raw + (sbase - raw);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sgen + OFF_ABORT);
+  uint32_t* tmem_ptr_smem = reinterpret_cast<uint32_t*>(sgen + OFF_TMEMPTR);
+  uint32_t* hcnt = reinterpret_cast<uint32_t*>(sgen + OFF_HCNT);
+  double* hmass = reinterpret_cast<double*>(sgen + OFF_HMASS);
+  float2* xch = reinterpret_cast<float2*>(sgen + OFF_XCH);
+  float2* rows_sm = reinterpret_cast<float2*>(sgen + OFF_ROW);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nbk = MODE == kHist1 ? kHistL1 : MODE == kHist2 ? kHistL2 : 1024;
+
+  if (threadIdx.x == 0) {
+    *abort_flag = dev::load_volatile(a.status) != 0 ? 1 : 0;
+    for (int s = 0; s < kStages; ++s) {
+      dev::mbar_init(bar_addr(sbase, B_KFULL + s), 1);
+      dev::mbar_init(bar_addr(sbase, B_KEMPTY + s), 1);
+    }
+    for (int x = 0; x < 2; ++x) {
+      dev::mbar_init(bar_addr(sbase, B_SFULL + x), 1);
+      dev::mbar_init(bar_addr(sbase, B_SEMPTY + x), 128);
+      dev::mbar_init(bar_addr(sbase, B_QFULL + x), 256);
+      dev::mbar_init(bar_addr(sbase, B_QEMPTY + x), 1);
+    }
+    dev::mbar_init(bar_addr(sbase, B_EPI), 256);
+    dev::mbar_init(bar_addr(sbase, B_DRAIN), 1);
+    dev::fence_mbar_init();
+  }
+  for (int i = threadIdx.x; i < kHistMax; i += kThreads) {
+    hcnt[i] = 0u;
+    hmass[i] = 0.0;
   }
   __syncthreads();
-  const int ty = tid >> 4, tx = tid & 15;
-  float acc[8][8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i)
-#pragma unroll
-    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
-#pragma unroll 2
-  for (int dd = 0; dd < kHeadDim; ++dd) {
-    const float* qd = qT + dd * kLStride;
-    const float* kd = kT + dd * kLStride;
-    const float4 q0 = *reinterpret_cast<const float4*>(qd + ty * 4);
-    const float4 q1 = *reinterpret_cast<const float4*>(qd + 64 + ty * 4);
-    const float4 k0 = *reinterpret_cast<const float4*>(kd + tx * 4);
-    const float4 k1 = *reinterpret_cast<const float4*>(kd + 64 + tx * 4);
-    const float qa[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-    const float ka[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-#pragma unroll
-      for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(qa[i], ka[j], acc[i][j]);
+  if (*abort_flag) return;   // an earlier kernel failed: do nothing (uniform, before TMEM is taken)
+  if (warp == 1) {
+    dev::tmem_alloc(dev::smem_u32(tmem_ptr_smem), kTmemCols);
+    dev::tmem_relinquish();
   }
-  // per row and 64-column half: max, sum of 2^(l - max) and min over the kept
-  // columns c <= r (the 16 threads of a row reduce by shuffles); then the row
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int r = r0 + (i >> 2) * 64 + ty * 4 + (i & 3);
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      float m = -INFINITY, mn = INFINITY;
-#pragma unroll
-      for (int jj = 0; jj < 4; ++jj) {
-        const int c = c0 + half * 64 + tx * 4 + jj;
-        if (c <= r) {
-          m = fmaxf(m, acc[i][half * 4 + jj]);
-          mn = fminf(mn, acc[i][half * 4 + jj]);
+  dev::tc_fence_before();
+  __syncthreads();
+  dev::tc_fence_after();
+  const uint32_t tmem = *tmem_ptr_smem;
+
+  if (warp < 4) dev::regs_release<kRegsControl>();
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    // the whole warp walks the stripes (tile masks); lane 0 issues the copies
+    if (lane == 0) {
+      dev::prefetch_tmap(&tm_khi);
+      dev::prefetch_tmap(&tm_klo);
+    }
+    int kt = 0;
+    bool ok = true;
+    PassCtx c;
+    int h, rt;
+    for (int it = 0; ok && item_of(a, blockIdx.x, it, h, rt); ++it) {
+      if (!head_live(a, MODE, h, c)) continue;
+      const uint64_t act = stripe_mask(a, c, h, rt, lane);
+      const int g = h / a.group;
+      for (int sw = 0; ok && sw < sweeps_of(MODE); ++sw) {
+        for (uint64_t m = act; ok && m; m &= m - 1) {
+          const int ct = __ffsll((long long)m) - 1;
+          const int s = kt % kStages;
+          if (lane == 0) {
+            ok = dev::mbar_wait(bar_addr(sbase, B_KEMPTY + s), ((kt / kStages) & 1) ^ 1, abort_flag, a.status, 41);
+            if (ok) {
+              const uint32_t bk = bar_addr(sbase, B_KFULL + s);
+              const uint32_t dst = sbase + OFF_K + s * 2 * kTileBytes;
+              dev::mbar_arrive_expect_tx(bk, 2 * kTileBytes);
+              dev::tma_load_3d(dst, &tm_khi, bk, 0, ct * 128, g);
+              dev::tma_load_3d(dst + kHalfBytes, &tm_khi, bk, 64, ct * 128, g);
+              dev::tma_load_3d(dst + kTileBytes, &tm_klo, bk, 0, ct * 128, g);
+              dev::tma_load_3d(dst + kTileBytes + kHalfBytes, &tm_klo, bk, 64, ct * 128, g);
+            }
+          }
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          if (ok) ++kt;
         }
       }
-#pragma unroll
-      for (int o = 1; o < 16; o <<= 1) {
-        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    }
+    if (!ok && lane == 0) {   // let the copies in flight land before the CTA exits
+      for (int s = 0; s < kStages && s < kt; ++s) {
+        const int last = kt - 1 - ((kt - 1 - s) % kStages);
+        dev::mbar_drain(bar_addr(sbase, B_KFULL + s), (last / kStages) & 1);
       }
-      float sum = 0.f;
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    // the whole warp walks the stripes; lane 0 issues every tcgen05.mma
+    const uint32_t idesc = dev::umma_idesc_bf16(128, 128, false);
+    int kt = 0, j = 0, qi = 0;
+    bool ok = true;
+    PassCtx c;
+    int h, rt;
+    for (int it = 0; ok && item_of(a, blockIdx.x, it, h, rt); ++it) {
+      if (!head_live(a, MODE, h, c)) continue;
+      const uint64_t act = stripe_mask(a, c, h, rt, lane);
+      if (act == 0) continue;
+      if (lane == 0) ok = dev::mbar_wait(bar_addr(sbase, B_QFULL + (qi & 1)), (qi >> 1) & 1, abort_flag, a.status, 42);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      dev::tc_fence_after();
+      const uint32_t qcol = tmem + 256u + (uint32_t)(qi & 1) * 128u;
+      for (int sw = 0; ok && sw < sweeps_of(MODE); ++sw) {
+        for (uint64_t m = act; ok && m; m &= m - 1) {
+          const int s = kt % kStages, buf = j & 1;
+          if (lane == 0) {
+            ok = dev::mbar_wait(bar_addr(sbase, B_KFULL + s), (kt / kStages) & 1, abort_flag, a.status, 43);
+            if (ok && j >= 2)
+              ok = dev::mbar_wait(bar_addr(sbase, B_SEMPTY + buf), ((j - 2) >> 1) & 1, abort_flag, a.status, 44);
+            if (ok) {
+              dev::tc_fence_after();
+              const uint32_t kh = sbase + OFF_K + s * 2 * kTileBytes, kl = kh + kTileBytes;
+              const uint32_t d = tmem + (uint32_t)buf * 128u;
 #pragma unroll
-      for (int jj = 0; jj < 4; ++jj) {
-        const int c = c0 + half * 64 + tx * 4 + jj;
-        if (c <= r) sum += dev::ex2(acc[i][half * 4 + jj] - m);
+              for (int kk = 0; kk < 8; ++kk)
+                dev::umma_ts(d, qcol + kk * 8, kmajor_desc(kh, kk), idesc, kk > 0 ? 1u : 0u);
+#pragma unroll
+              for (int kk = 0; kk < 8; ++kk) dev::umma_ts(d, qcol + 64 + kk * 8, kmajor_desc(kh, kk), idesc, 1u);
+#pragma unroll
+              for (int kk = 0; kk < 8; ++kk) dev::umma_ts(d, qcol + kk * 8, kmajor_desc(kl, kk), idesc, 1u);
+              dev::umma_commit(bar_addr(sbase, B_SFULL + buf));
+              dev::umma_commit(bar_addr(sbase, B_KEMPTY + s));
+            }
+          }
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          ++kt;
+          ++j;
+        }
       }
+      if (lane == 0) dev::umma_commit(bar_addr(sbase, B_QEMPTY + (qi & 1)));   // this stripe's Q-bar is no longer read
+      ++qi;
+    }
+    if (lane == 0) {   // every MMA issued completes before TMEM is released
+      dev::umma_commit(bar_addr(sbase, B_DRAIN));
+      dev::mbar_drain(bar_addr(sbase, B_DRAIN), 0);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ---------------------------------------------------------------- epilogue warpgroups
+    dev::regs_acquire<kRegsEpilogue>();
+    const int wg = (warp - 4) >> 2;               // 0 or 1: the tiles j with j % 2 == wg
+    const int quarter = warp & 3;                 // TMEM lane quarter of this warp
+    const int lr = quarter * 32 + lane;           // row inside the tile
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    uint32_t epi_phase = 0;
+    int j = 0, qi = 0;
+    bool ok = true;
+    PassCtx c;
+    int h, rt;
+
+    // write the Q-bar rows of stripe (hq, rtq) into TMEM buffer `buf` (this
+    // warpgroup's half: hi for warpgroup 0, lo for 1); q = its index among the
+    // stripes with tensor-core work
+    auto write_q = [&](int hq, int rtq, int q) -> bool {
+      const int buf = q & 1;
+      if (q >= 2 && !warp_wait(bar_addr(sbase, B_QEMPTY + buf), ((q - 2) >> 1) & 1, abort_flag, a.status, 45))
+        return false;
+      dev::tc_fence_after();
+      const int r = rtq * 128 + lr;
+      const __nv_bfloat16* src = (wg == 0 ? a.qhi : a.qlo) + ((size_t)hq * a.nb + r) * kHeadDim;
+      const uint32_t col = tmem + lane_base + 256u + (uint32_t)buf * 128u + (uint32_t)wg * 64u;
 #pragma unroll
-      for (int o = 1; o < 16; o <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-      const int c64 = 2 * ct + half;   // statistics tile of this half
-      if (tx == 0 && r < a.nb && c64 * kLT < a.nb && c64 * kLT <= r)
-        a.tri_stats[((size_t)h * a.nb + r) * a.n_ct + c64] = make_float4(m, sum, mn, 0.f);
-    }
-    if (r >= a.nb) continue;
-    float* row = a.tri_buf + (size_t)h * a.tri_stride + tri_off(r);
+      for (int part = 0; part < 4; ++part) {
+        uint32_t w[16];
+        if (r < a.nb) {
+          const uint4* p = reinterpret_cast<const uint4*>(src + part * 32);
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int c = c0 + (j >> 2) * 64 + tx * 4 + (j & 3);
-      if (c <= r) row[c] = acc[i][j];
-    }
-  }
-}
-
-// A grid-stride loop over (query head, triangle tile) items: heads not
-// routed PE cost one iteration, not a CTA launch (a launched CTA reserves
-// 132 KB of shared memory, one per SM, even when it exits at once).
-__global__ void __launch_bounds__(256) pe_logits_kernel(PeArgs a, int n_tri_tiles) {
-  extern __shared__ __align__(16) float lsm[];
-  for (long long item = blockIdx.x; item < (long long)a.h_q * n_tri_tiles; item += gridDim.x) {
-    const int h = (int)(item / n_tri_tiles);
-    if (a.route[h] != 1) continue;   // uniform over the CTA
-    __syncthreads();                 // the previous item's reads of lsm are done
-    pe_logits_tile(a, h, (int)(item % n_tri_tiles), lsm);
-  }
-}
-
-__device__ __forceinline__ void hist_flush(PeHist* hist, uint32_t bucket, unsigned long long cnt, double mass) {
-  if (cnt == 0) return;
-  atomicAdd(&hist->count[bucket], cnt);
-  atomicAdd(&hist->mass[bucket], mass);
-}
-
-constexpr int kRowsPerCta = 8;  // one warp per row
-// Level-0 buckets (bits 31..20) of the values in [0, 1): every entry of the
-// normalised map is at most 1 / N_b, so its bucket is below 0x3F8.
-constexpr int kL0Low = 1024;
-
-constexpr int kWin = 64;   // level-0 buckets of a row's window in the per-warp histogram
-
-// Row softmax of the pooled logits, divided by N_b (the flattened map's
-// total), written in place; level-0 histogram (bits 31..20) with float64
-// mass. One warp per row; the row maximum and normaliser come from the
-// logits kernel's per-tile statistics, so the row is read once. Each lane
-// merges runs of equal buckets; a row whose values span fewer than kWin
-// buckets gathers them in its warp's own window (lanes of one warp mostly
-// hit one bucket, so windows keep contention inside a warp), a wider row
-// (a heavy-tailed map) in the CTA's histogram of all level-0 buckets below
-// 1.0. Non-empty buckets reach the global histogram with one atomic each.
-__global__ void __launch_bounds__(256) pe_softmax_kernel(PeArgs a) {
-  const int h = blockIdx.y;
-  if (a.route[h] != 1) return;   // uniform over the CTA
-  __shared__ unsigned long long scount[kL0Low];
-  __shared__ double smass[kL0Low];
-  __shared__ unsigned long long wcount[kRowsPerCta][kWin];
-  __shared__ double wmass[kRowsPerCta][kWin];
-  for (int i = threadIdx.x; i < kL0Low; i += blockDim.x) {
-    scount[i] = 0;
-    smass[i] = 0.0;
-  }
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int i = lane; i < kWin; i += 32) {
-    wcount[warp][i] = 0;
-    wmass[warp][i] = 0.0;
-  }
-  __syncthreads();
-  const int r = blockIdx.x * kRowsPerCta + warp;
-  PeHist* hist = a.hist + h;
-  uint32_t b_lo = 0;
-  bool window = false;
-  if (r < a.nb) {
-    float* row = a.tri_buf + (size_t)h * a.tri_stride + tri_off(r);
-    // row maximum and normaliser from the logits kernel's per-tile statistics
-    const float4* st = a.tri_stats + ((size_t)h * a.nb + r) * a.n_ct;
-    const int n_t = r / kLT + 1;   // column tiles holding c <= r
-    float m = -INFINITY, mn = INFINITY;
-    for (int i = lane; i < n_t; i += 32) {
-      m = fmaxf(m, st[i].x);
-      mn = fminf(mn, st[i].z);
-    }
-    m = warp_max(m);
-    mn = warp_min(mn);
-    float s = 0.f;
-    for (int i = lane; i < n_t; i += 32) {
-      const float4 e = st[i];
-      s += e.y * dev::ex2(e.x - m);
-    }
-    s = warp_sum(s);
-    const float inv = 1.f / (s * (float)a.nb);
-    const uint32_t b_hi = __float_as_uint(inv) >> 20;                       // bucket of the row maximum
-    b_lo = __float_as_uint(dev::ex2(mn - m) * inv) >> 20;                   // bucket of the row minimum
-    window = b_hi >= b_lo && b_hi - b_lo < (uint32_t)kWin;
-    uint32_t cur = 0xffffffffu;
-    unsigned long long cnt = 0;
-    double mass = 0.0;
-    auto flush = [&]() {
-      if (!cnt) return;
-      if (window) {
-        atomicAdd(&wcount[warp][cur - b_lo], cnt);
-        atomicAdd(&wmass[warp][cur - b_lo], mass);
-      } else if (cur < (uint32_t)kL0Low) {
-        atomicAdd(&scount[cur], cnt);
-        atomicAdd(&smass[cur], mass);
-      } else {
-        hist_flush(hist, cur, cnt, mass);
+          for (int x = 0; x < 4; ++x) {
+            const uint4 u = p[x];
+            w[4 * x] = u.x;
+            w[4 * x + 1] = u.y;
+            w[4 * x + 2] = u.z;
+            w[4 * x + 3] = u.w;
+          }
+        } else {
+#pragma unroll
+          for (int x = 0; x < 16; ++x) w[x] = 0u;
+        }
+        dev::tmem_st16(col + part * 16, w);
       }
+      dev::tmem_wait_st();
+      dev::tc_fence_before();
+      dev::mbar_arrive(bar_addr(sbase, B_QFULL + buf));
+      return true;
     };
-    for (int c = lane; c <= r; c += 32) {
-      const float v = dev::ex2(row[c] - m) * inv;
-      row[c] = v;
-      const uint32_t bucket = __float_as_uint(v) >> 20;
-      if (bucket != cur) {
-        flush();
-        cur = bucket;
-        cnt = 0;
-        mass = 0.0;
+    // next stripe after item `it` with tensor-core work, for the Q prefetch
+    auto next_active = [&](int it, int& hn, int& rtn) -> bool {
+      PassCtx cn;
+      for (int k = it + 1; item_of(a, blockIdx.x, k, hn, rtn); ++k)
+        if (head_live(a, MODE, hn, cn) && stripe_mask(a, cn, hn, rtn, lane) != 0) return true;
+      return false;
+    };
+    // one S tile into registers (and the buffer released)
+    auto load_s = [&](float (&s)[128]) -> bool {
+      const int buf = j & 1;
+      if (!warp_wait(bar_addr(sbase, B_SFULL + buf), (j >> 1) & 1, abort_flag, a.status, 46)) return false;
+      dev::tc_fence_after();
+      dev::tmem_ld128(tmem + lane_base + (uint32_t)buf * 128u, s);
+      dev::tmem_wait_ld();
+      dev::tc_fence_before();
+      dev::mbar_arrive(bar_addr(sbase, B_SEMPTY + buf));
+      return true;
+    };
+    auto flush_hist = [&](int hh) -> bool {
+      if (!epi_sync(sbase, epi_phase, abort_flag, a.status)) return false;
+      PeHist* gh = a.hist + hh;
+      for (int i = threadIdx.x - 128; i < nbk; i += 256) {
+        const uint32_t cnt = hcnt[i];
+        if (cnt) {
+          atomicAdd(&gh->count[i], (unsigned long long)cnt);
+          atomicAdd(&gh->mass[i], hmass[i]);
+          hcnt[i] = 0u;
+          hmass[i] = 0.0;
+        }
       }
-      ++cnt;
-      mass += (double)v;
+      return epi_sync(sbase, epi_phase, abort_flag, a.status);
+    };
+
+    {   // the first stripe with tensor-core work
+      int h0, rt0;
+      if (next_active(-1, h0, rt0)) ok = write_q(h0, rt0, 0);
     }
-    flush();
+    for (int it = 0; ok && item_of(a, blockIdx.x, it, h, rt); ++it) {
+      if (!head_live(a, MODE, h, c)) continue;
+      const uint64_t act_mask = stripe_mask(a, c, h, rt, lane);
+      const uint64_t above_mask = (MODE == kMask && !c.all) ? stripe_above(a, c, h, rt, lane) : 0ull;
+      const int n_act = __popcll(act_mask);
+      if (n_act > 0) {
+        int hn, rtn;
+        if (next_active(it, hn, rtn) && !write_q(hn, rtn, qi + 1)) {
+          ok = false;
+          break;
+        }
+      }
+      const int r = rt * 128 + lr;
+      const bool row_ok = r < a.nb;
+      const int ncol = row_ok ? r - rt * 128 : -1;     // last valid column of the diagonal tile
+      // last valid column of tile ct: every column before the diagonal tile
+      // (c <= r < N_b), up to the diagonal in it, none in a padding row
+      auto last_of = [&](int ct) { return !row_ok ? -1 : (ct < rt ? 127 : ncol); };
+      float s[128];
+      if (MODE == kStatsHist0) {
+        // sweep 1: this warpgroup's tiles, online maximum and normaliser per row
+        float m = -INFINITY, l = 0.f;
+        for (int ct = 0; ct <= rt; ++ct, ++j) {
+          if ((j & 1) != wg) continue;
+          if (!load_s(s)) {
+            ok = false;
+            break;
+          }
+          const int last = last_of(ct);
+          float tmax = -INFINITY;
+#pragma unroll
+          for (int cc = 0; cc < 128; ++cc) tmax = cc <= last ? fmaxf(tmax, s[cc]) : tmax;
+          if (tmax > m) {
+            l *= dev::ex2(m - tmax);
+            m = tmax;
+          }
+          float sum = 0.f;
+#pragma unroll
+          for (int cc = 0; cc < 128; ++cc) sum += cc <= last ? dev::ex2(s[cc] - m) : 0.f;
+          l += sum;
+        }
+        if (!ok) break;
+        // the two warpgroups' statistics of each row, combined
+        if (wg == 1) xch[lr] = make_float2(m, l);
+        if (!epi_sync(sbase, epi_phase, abort_flag, a.status)) {
+          ok = false;
+          break;
+        }
+        if (wg == 0) {
+          const float2 o = xch[lr];
+          const float M = fmaxf(m, o.x);
+          const float L = (m == -INFINITY ? 0.f : l * dev::ex2(m - M)) + (o.x == -INFINITY ? 0.f : o.y * dev::ex2(o.x - M));
+          const float2 st = make_float2(M, 1.f / (L * (float)a.nb));
+          rows_sm[lr] = st;
+          if (row_ok) a.row_stat[(size_t)h * a.nb + r] = st;
+        }
+        if (!epi_sync(sbase, epi_phase, abort_flag, a.status)) {
+          ok = false;
+          break;
+        }
+        const float2 st = rows_sm[lr];
+        // sweep 2: entries, level-0 histogram (runs of equal buckets merged), tile key ranges
+        for (int ct = 0; ct <= rt; ++ct, ++j) {
+          if ((j & 1) != wg) continue;
+          if (!load_s(s)) {
+            ok = false;
+            break;
+          }
+          const int last = last_of(ct);
+          uint32_t kmin = 0xFFFFFFFFu, kmax = 0u, cur = 0xFFFFFFFFu, cnt = 0u;
+          double mass = 0.0;
+#pragma unroll
+          for (int cc = 0; cc < 128; ++cc) {
+            if (cc > last) continue;
+            const float v = entry_value(s[cc], st.x, st.y);
+            const uint32_t key = __float_as_uint(v);
+            kmin = min(kmin, key);
+            kmax = max(kmax, key);
+            const uint32_t b = key >> 20;
+            if (b != cur) {
+              if (cnt) hist_add(hcnt, hmass, cur, cnt, mass);
+              cur = b;
+              cnt = 0u;
+              mass = 0.0;
+            }
+            ++cnt;
+            mass += (double)v;
+          }
+          if (cnt) hist_add(hcnt, hmass, cur, cnt, mass);
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) {
+            kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+            kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+          }
+          if (lane == 0) a.tile_kr[(((size_t)h * a.nt + rt) * a.nt + ct) * 4 + quarter] = make_uint2(kmin, kmax);
+        }
+        if (!ok) break;
+        if (!flush_hist(h)) {
+          ok = false;
+          break;
+        }
+      } else {
+        const float2 st = row_ok ? a.row_stat[(size_t)h * a.nb + r] : make_float2(0.f, 0.f);
+        uint32_t* mrow = a.pe_mask + ((size_t)h * a.nb + (row_ok ? r : 0)) * a.words;
+        uint32_t* trow = a.tie_cnt + ((size_t)h * a.nb + (row_ok ? r : 0)) * a.nt;
+        unsigned long long kept = 0;
+        for (int ct = 0; ct <= rt; ++ct) {
+          const bool act = (act_mask >> ct) & 1ull;
+          const int last = last_of(ct);
+          const int owner = act ? (j & 1) : (ct & 1);
+          if (owner != wg || (!act && (MODE == kHist1 || MODE == kHist2))) {
+            if (act) ++j;
+            continue;
+          }
+          if (act) {
+            if (!load_s(s)) {
+              ok = false;
+              break;
+            }
+            ++j;
+          }
+          if (MODE == kHist1 || MODE == kHist2) {
+            const int shift_p = MODE == kHist1 ? 20 : 8;
+            const int shift_b = MODE == kHist1 ? 8 : 0;
+            const uint32_t bmask = MODE == kHist1 ? 0xFFFu : 0xFFu;
+#pragma unroll
+            for (int cc = 0; cc < 128; ++cc) {
+              if (cc > last) continue;
+              const float v = entry_value(s[cc], st.x, st.y);
+              const uint32_t key = __float_as_uint(v);
+              if ((key >> shift_p) == c.prefix) hist_add(hcnt, hmass, (key >> shift_b) & bmask, 1u, (double)v);
+            }
+          } else if (MODE == kTies) {
+            uint32_t ties = 0;
+            if (act) {
+#pragma unroll
+              for (int cc = 0; cc < 128; ++cc) {
+                if (cc > last) continue;
+                ties += __float_as_uint(entry_value(s[cc], st.x, st.y)) == c.cut ? 1u : 0u;
+              }
+            }
+            if (row_ok) trow[ct] = ties;
+          } else {   // kMask
+            uint32_t w[4] = {0u, 0u, 0u, 0u};
+            if (row_ok) {
+              if (c.all || ((above_mask >> ct) & 1ull)) {   // every entry kept
+#pragma unroll
+                for (int cc = 0; cc < 128; ++cc)
+                  if (cc <= last) w[cc >> 5] |= 1u << (cc & 31);
+              } else if (act) {
+                unsigned long long rank = c.partial_ties ? trow[ct] : 0ull;
+#pragma unroll
+                for (int cc = 0; cc < 128; ++cc) {
+                  if (cc > last) continue;
+                  const uint32_t key = __float_as_uint(entry_value(s[cc], st.x, st.y));
+                  bool keep = key > c.cut || (ct == rt && cc == last);
+                  if (key == c.cut) {
+                    keep = keep || !c.partial_ties || rank < c.t_keep;
+                    ++rank;
+                  }
+                  if (keep) w[cc >> 5] |= 1u << (cc & 31);
+                }
+              }
+              if (ct == rt) w[ncol >> 5] |= 1u << (ncol & 31);   // the diagonal block
+#pragma unroll
+              for (int x = 0; x < 4; ++x) {
+                const int word = ct * 4 + x;
+                if (word < a.words) {
+                  mrow[word] = w[x];
+                  kept += __popc(w[x]);
+                }
+              }
+            }
+          }
+        }
+        if (!ok) break;
+        if (MODE == kHist1 || MODE == kHist2) {
+          if (!flush_hist(h)) {
+            ok = false;
+            break;
+          }
+        }
+        if (MODE == kMask) {
+          // words of the columns beyond this stripe's diagonal tile are zero
+          if (wg == 0 && row_ok)
+            for (int word = (rt + 1) * 4; word < a.words; ++word) mrow[word] = 0u;
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) kept += __shfl_xor_sync(0xffffffffu, kept, o);
+          if (lane == 0 && kept) atomicAdd(reinterpret_cast<unsigned long long*>(a.pe_count + h), kept);
+          if (rt == 0 && wg == 0 && lr == 0) a.pe_cut[h] = c.all ? 0.f : __uint_as_float(c.cut);
+        }
+      }
+      if (n_act > 0) ++qi;
+    }
+    dev::tc_fence_before();
   }
   __syncthreads();
-  if (window) {   // the warp's window into the global histogram
-    for (int i = lane; i < kWin; i += 32)
-      if (wcount[warp][i]) hist_flush(hist, b_lo + (uint32_t)i, wcount[warp][i], wmass[warp][i]);
+  if (warp == 1) {
+    dev::tc_fence_after();
+    dev::tmem_dealloc(tmem, kTmemCols);
   }
-  for (int i = threadIdx.x; i < kL0Low; i += blockDim.x)
-    if (scount[i]) hist_flush(hist, (uint32_t)i, scount[i], smass[i]);
 }
 
-// Histogram of the entries whose key matches the prefix found so far
-// (level 1: bits 19..8 under the 12-bit prefix; level 2: bits 7..0 under the
-// 24-bit prefix). float4 sweeps over the head's triangle (stride padded to
-// 64); each CTA gathers its part in shared memory (dynamic, 16 bytes per
-// bucket) and adds its non-empty buckets to the global histogram.
-__global__ void __launch_bounds__(256) pe_hist_kernel(PeArgs a, int level) {
-  const int h = blockIdx.y;
-  if (a.route[h] != 1) return;
-  const PeState* st = a.state + h;
-  if (st->all) return;   // uniform over the CTA
-  extern __shared__ __align__(16) unsigned char hsm[];
-  const int nbk = level == 1 ? kHistL1 : kHistL2;
-  unsigned long long* scount = reinterpret_cast<unsigned long long*>(hsm);
-  double* smass = reinterpret_cast<double*>(hsm + (size_t)nbk * sizeof(unsigned long long));
-  for (int i = threadIdx.x; i < nbk; i += blockDim.x) {
-    scount[i] = 0;
-    smass[i] = 0.0;
-  }
-  __syncthreads();
-  const uint32_t prefix = st->prefix;
-  const int shift_p = level == 1 ? 20 : 8;
-  const int shift_b = level == 1 ? 8 : 0;
-  const uint32_t bmask = level == 1 ? 0xFFFu : 0xFFu;
-  const float4* tri4 = reinterpret_cast<const float4*>(a.tri_buf + (size_t)h * a.tri_stride);
-  const long long n4 = (a.tri + 3) / 4;
-  for (long long p = (long long)blockIdx.x * blockDim.x + threadIdx.x; p < n4; p += (long long)gridDim.x * blockDim.x) {
-    const float4 v4 = tri4[p];
-    const float vv[4] = {v4.x, v4.y, v4.z, v4.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      if (4 * p + i >= a.tri) break;
-      const uint32_t key = __float_as_uint(vv[i]);
-      if ((key >> shift_p) == prefix) {
-        const uint32_t b = (key >> shift_b) & bmask;
-        atomicAdd(&scount[b], 1ull);
-        atomicAdd(&smass[b], (double)vv[i]);
-      }
-    }
-  }
-  __syncthreads();
-  PeHist* hist = a.hist + h;
-  for (int i = threadIdx.x; i < nbk; i += blockDim.x)
-    if (scount[i]) hist_flush(hist, (uint32_t)i, scount[i], smass[i]);
-}
+// ------------------------------------------------------------------ the cut
 
 // Walk the buckets of the current level from the largest key down, carrying
 // the mass above; pick the bucket where the cumulative mass reaches gamma.
@@ -387,6 +767,9 @@ __global__ void __launch_bounds__(1024) pe_find_kernel(PeArgs a, int level) {
       st->s_above = 0.0;
       st->prefix = 0;
       st->all = a.gamma >= 1.f ? 1u : 0u;
+      st->n_ties = 0;
+      st->t_keep = 0;
+      st->cut_key = 0;
     }
     s_found = 0;
   }
@@ -400,8 +783,7 @@ __global__ void __launch_bounds__(1024) pe_find_kernel(PeArgs a, int level) {
   }
   tsum[tid] = my;
   __syncthreads();
-  // inclusive scan over threads (descending bucket order)
-  for (int off = 1; off < 1024; off <<= 1) {
+  for (int off = 1; off < 1024; off <<= 1) {   // inclusive scan over threads (descending bucket order)
     const double v = tid >= off ? tsum[tid - off] : 0.0;
     __syncthreads();
     tsum[tid] += v;
@@ -478,94 +860,48 @@ __global__ void __launch_bounds__(1024) pe_find_kernel(PeArgs a, int level) {
   }
 }
 
-// Ties needed in part only: count entries equal to the cut value per row (one warp per row).
-__global__ void __launch_bounds__(256) pe_tie_count_kernel(PeArgs a) {
-  const int h = blockIdx.y;
-  if (a.route[h] != 1) return;
-  const PeState* st = a.state + h;
-  if (st->all || st->t_keep >= st->n_ties) return;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int r = blockIdx.x * kRowsPerCta + warp;
-  if (r >= a.nb) return;
-  const float* row = a.tri_buf + (size_t)h * a.tri_stride + tri_off(r);
-  uint32_t cnt = 0;
-  for (int c = lane; c <= r; c += 32) cnt += (__float_as_uint(row[c]) == st->cut_key) ? 1u : 0u;
-  for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
-  if (lane == 0) a.tie_rows[(size_t)h * a.nb + r] = cnt;
-}
-
-// Exclusive scan of the per-row tie counts (one CTA of 1024 threads per head).
+// Exclusive scan, in flat order (row by row, tiles left to right), of the
+// per-(row, tile) tie counts of heads whose cut keeps part of its ties.
+// One CTA of 1024 threads per head; entries (r, ct) with ct > r / 128 hold
+// nothing and are not read.
 __global__ void __launch_bounds__(1024) pe_tie_scan_kernel(PeArgs a) {
   const int h = blockIdx.x;
   if (a.route[h] != 1) return;
   const PeState* st = a.state + h;
   if (st->all || st->t_keep >= st->n_ties) return;
-  __shared__ uint32_t part[1024];
-  uint32_t* rows = a.tie_rows + (size_t)h * a.nb;
+  __shared__ unsigned long long part[1024];
+  uint32_t* cnt = a.tie_cnt + (size_t)h * a.nb * a.nt;
   const int per = (a.nb + 1023) / 1024;
   const int lo = threadIdx.x * per, hi = min(a.nb, lo + per);
-  uint32_t s = 0;
-  for (int r = lo; r < hi; ++r) s += rows[r];
+  unsigned long long s = 0;
+  for (int r = lo; r < hi; ++r)
+    for (int ct = 0; ct <= r / 128; ++ct) s += cnt[(size_t)r * a.nt + ct];
   part[threadIdx.x] = s;
   __syncthreads();
   for (int off = 1; off < 1024; off <<= 1) {
-    const uint32_t v = threadIdx.x >= off ? part[threadIdx.x - off] : 0u;
+    const unsigned long long v = threadIdx.x >= off ? part[threadIdx.x - off] : 0ull;
     __syncthreads();
     part[threadIdx.x] += v;
     __syncthreads();
   }
-  uint32_t acc = threadIdx.x > 0 ? part[threadIdx.x - 1] : 0u;
-  for (int r = lo; r < hi; ++r) {
-    const uint32_t v = rows[r];
-    rows[r] = acc;
-    acc += v;
-  }
+  unsigned long long acc = threadIdx.x > 0 ? part[threadIdx.x - 1] : 0ull;
+  for (int r = lo; r < hi; ++r)
+    for (int ct = 0; ct <= r / 128; ++ct) {
+      uint32_t* e = cnt + (size_t)r * a.nt + ct;
+      const uint32_t v = *e;
+      // offsets beyond 2^32 cannot occur: a head has at most 2^25 causal blocks
+      *e = (uint32_t)acc;
+      acc += v;
+    }
 }
 
-// Write the PE mask row by row (one warp per row): keep (r, c), c <= r, when
-// its value is above the cut, or equal to it and among the first t_keep ties
-// in flat order, or c == r; or everything when the cut keeps all.
-__global__ void __launch_bounds__(256) pe_mask_kernel(PeArgs a) {
-  const int h = blockIdx.y;
-  if (a.route[h] != 1) return;
-  const PeState* st = a.state + h;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int r = blockIdx.x * kRowsPerCta + warp;
-  __shared__ unsigned long long kept_cta;
-  if (threadIdx.x == 0) kept_cta = 0;
-  __syncthreads();
-  if (r < a.nb) {
-    const bool all = st->all != 0;
-    const uint32_t cut = st->cut_key;
-    const bool partial_ties = !all && st->t_keep < st->n_ties;
-    const unsigned long long t_keep = st->t_keep;
-    unsigned long long tie_base = partial_ties ? a.tie_rows[(size_t)h * a.nb + r] : 0ull;
-    const float* row = a.tri_buf + (size_t)h * a.tri_stride + tri_off(r);
-    uint32_t* mrow = a.pe_mask + ((size_t)h * a.nb + r) * a.words;
-    uint32_t kept = 0;
-    for (int w = 0; w < a.words; ++w) {
-      const int c = w * 32 + lane;
-      int keep = 0, tie = 0;
-      if (c <= r) {
-        const uint32_t key = __float_as_uint(row[c]);
-        tie = (!all && key == cut) ? 1 : 0;
-        keep = all || c == r || key > cut || (tie && !partial_ties);
-      }
-      if (partial_ties) {
-        const unsigned tb = __ballot_sync(0xffffffffu, tie);
-        const unsigned long long rank = tie_base + __popc(tb & ((1u << lane) - 1u));
-        if (tie && rank < t_keep) keep = 1;
-        tie_base += __popc(tb);
-      }
-      const unsigned bal = __ballot_sync(0xffffffffu, keep);
-      if (lane == 0) mrow[w] = bal;
-      kept += __popc(bal);
-    }
-    if (lane == 0) atomicAdd(&kept_cta, (unsigned long long)kept);
-    if (lane == 0 && r == 0) a.pe_cut[h] = all ? 0.f : __uint_as_float(cut);
-  }
-  __syncthreads();
-  if (threadIdx.x == 0 && kept_cta) atomicAdd(reinterpret_cast<unsigned long long*>(a.pe_count + h), kept_cta);
+template <int MODE>
+cudaError_t launch_sweep(const CUtensorMap& mh, const CUtensorMap& ml, const PeArgs& a, int grid, cudaStream_t st) {
+  cudaError_t e = cudaFuncSetAttribute(pe_sweep_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       kSmemBytes);
+  if (e != cudaSuccess) return e;
+  pe_sweep_kernel<MODE><<<grid, kThreads, kSmemBytes, st>>>(mh, ml, a);
+  return cudaGetLastError();
 }
 
 }  // namespace
@@ -573,70 +909,62 @@ __global__ void __launch_bounds__(256) pe_mask_kernel(PeArgs a) {
 cudaError_t launch_pe(const void* q, const void* k, const Shape& s, char* ws, const WsLayout& L,
                       const IndexPtrs& ix, cudaStream_t st) {
   PeArgs a;
-  a.n = s.n;
   a.nb = s.nb;
+  a.nt = (s.nb + 127) / 128;
   a.words = s.words;
   a.group = s.group;
   a.h_q = s.h_q;
-  a.h_kv = s.h_kv;
-  a.tri = s.tri;
-  a.tri_stride = s.tri_stride;
-  a.scale_log2 = s.scale_log2;
   a.gamma = s.gamma;
   a.route = ix.route;
-  a.kv_pe = reinterpret_cast<const int32_t*>(ws + L.kv_pe);
-  a.qbar = reinterpret_cast<float*>(ws + L.qbar);
-  a.kbar = reinterpret_cast<float*>(ws + L.kbar);
-  a.tri_buf = reinterpret_cast<float*>(ws + L.tri);
-  a.tri_stats = reinterpret_cast<float4*>(ws + L.tri_stats);
-  a.n_ct = (s.nb + kLT - 1) / kLT;
+  auto* qhi = reinterpret_cast<__nv_bfloat16*>(ws + L.qhi);
+  auto* qlo = reinterpret_cast<__nv_bfloat16*>(ws + L.qlo);
+  auto* khi = reinterpret_cast<__nv_bfloat16*>(ws + L.khi);
+  auto* klo = reinterpret_cast<__nv_bfloat16*>(ws + L.klo);
+  a.qhi = qhi;
+  a.qlo = qlo;
+  a.row_stat = reinterpret_cast<float2*>(ws + L.row_stat);
+  a.tile_kr = reinterpret_cast<uint2*>(ws + L.tile_kr);
+  a.tie_cnt = reinterpret_cast<uint32_t*>(ws + L.tie_cnt);
   a.hist = reinterpret_cast<PeHist*>(ws + L.hist);
   a.state = reinterpret_cast<PeState*>(ws + L.pe_state);
-  a.tie_rows = reinterpret_cast<uint32_t*>(ws + L.tie_rows);
   a.pe_mask = ix.pe_mask;
   a.pe_count = ix.pe_count;
   a.pe_cut = ix.pe_cut;
   a.status = reinterpret_cast<int32_t*>(ws + L.status);
+  const int32_t* kv_pe = reinterpret_cast<const int32_t*>(ws + L.kv_pe);
+
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
 
   cudaError_t e = cudaMemsetAsync(a.hist, 0, sizeof(PeHist) * s.h_q, st);
   if (e != cudaSuccess) return e;
-  // the query-head pooling is gated by the route (1 = PE); the key pooling
-  // by the per-group PE flag
-  if (s.fp32) {
-    pool_kernel<float><<<dim3(s.nb, s.h_q), 128, 0, st>>>(static_cast<const float*>(q), a.qbar, s.n, s.nb, ix.route);
-    pool_kernel<float><<<dim3(s.nb, s.h_kv), 128, 0, st>>>(static_cast<const float*>(k), a.kbar, s.n, s.nb, a.kv_pe);
-  } else {
-    pool_kernel<__nv_bfloat16><<<dim3(s.nb, s.h_q), 128, 0, st>>>(static_cast<const __nv_bfloat16*>(q), a.qbar,
-                                                                  s.n, s.nb, ix.route);
-    pool_kernel<__nv_bfloat16><<<dim3(s.nb, s.h_kv), 128, 0, st>>>(static_cast<const __nv_bfloat16*>(k), a.kbar,
-                                                                   s.n, s.nb, a.kv_pe);
-  }
-  const size_t lsmem = 2 * kHeadDim * kLStride * sizeof(float);
-  e = cudaFuncSetAttribute(pe_logits_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lsmem);
-  if (e != cudaSuccess) return e;
-  const int nt = (s.nb + kLT2 - 1) / kLT2;
-  {
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int n_tri_tiles = nt * (nt + 1) / 2;
-    const long long items = (long long)s.h_q * n_tri_tiles;
-    pe_logits_kernel<<<(int)std::min<long long>(items, sms), 256, lsmem, st>>>(a, n_tri_tiles);
-  }
-  const int row_ctas = (s.nb + kRowsPerCta - 1) / kRowsPerCta;
-  pe_softmax_kernel<<<dim3(row_ctas, s.h_q), 256, 0, st>>>(a);
+  const int pool_grid = 4 * sms;
+  if (s.fp32)
+    pe_pool_kernel<float><<<pool_grid, kPoolThreads, 0, st>>>(static_cast<const float*>(q),
+                                                              static_cast<const float*>(k), s.n, s.nb, a.nt * 128,
+                                                              s.h_q, s.h_kv, s.scale_log2, ix.route, kv_pe, qhi, qlo,
+                                                              khi, klo);
+  else
+    pe_pool_kernel<__nv_bfloat16><<<pool_grid, kPoolThreads, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), s.n, s.nb, a.nt * 128, s.h_q,
+        s.h_kv, s.scale_log2, ix.route, kv_pe, qhi, qlo, khi, klo);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+  CUtensorMap mh, ml;
+  if (!make_bf16_map(&mh, khi, a.nt * 128, s.h_kv, 128) || !make_bf16_map(&ml, klo, a.nt * 128, s.h_kv, 128))
+    return cudaErrorInvalidValue;
+  // one CTA per SM, at most one per stripe
+  const int grid = (int)std::min<long long>(sms, (long long)s.h_q * a.nt);
+  if ((e = launch_sweep<kStatsHist0>(mh, ml, a, grid, st)) != cudaSuccess) return e;
   pe_find_kernel<<<s.h_q, 1024, 0, st>>>(a, 0);
-  const int hist_ctas = (int)std::min<long long>(296, (s.tri / 4 + 255) / 256 + 1);
-  const size_t hsm1 = (size_t)kHistL1 * 16, hsm2 = (size_t)kHistL2 * 16;
-  e = cudaFuncSetAttribute(pe_hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hsm1);
-  if (e != cudaSuccess) return e;
-  pe_hist_kernel<<<dim3(hist_ctas, s.h_q), 256, hsm1, st>>>(a, 1);
+  if ((e = launch_sweep<kHist1>(mh, ml, a, grid, st)) != cudaSuccess) return e;
   pe_find_kernel<<<s.h_q, 1024, 0, st>>>(a, 1);
-  pe_hist_kernel<<<dim3(hist_ctas, s.h_q), 256, hsm2, st>>>(a, 2);
+  if ((e = launch_sweep<kHist2>(mh, ml, a, grid, st)) != cudaSuccess) return e;
   pe_find_kernel<<<s.h_q, 1024, 0, st>>>(a, 2);
-  pe_tie_count_kernel<<<dim3(row_ctas, s.h_q), 256, 0, st>>>(a);
+  if ((e = launch_sweep<kTies>(mh, ml, a, grid, st)) != cudaSuccess) return e;
   pe_tie_scan_kernel<<<s.h_q, 1024, 0, st>>>(a);
-  pe_mask_kernel<<<dim3(row_ctas, s.h_q), 256, 0, st>>>(a);
+  if ((e = launch_sweep<kMask>(mh, ml, a, grid, st)) != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

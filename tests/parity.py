@@ -5,7 +5,11 @@
 * VS masks: bit-exact, except a block whose oracle mass lies within 1e-3
   relative of alpha*mu (a flip).
 * PE masks: bit-exact, except an entry whose oracle value lies within 1e-3
-  relative of the oracle's cut value (a flip).
+  relative of the oracle's cut value, or whose place in the oracle's sorted
+  order has a cumulative mass (of the entries before it) within 1e-3
+  relative of gamma: Algorithm 4's threshold is gamma on that cumulative sum,
+  so an entry sitting on it (for instance when whole rows' mass adds up to
+  gamma exactly) is decided by rounding either way (a flip).
 * Outputs on the same indices: two normalisations of the max error, each
   within 2e-2 (bf16) or 1e-4 (fp32):
   - per head: max |o - o_ref| / max |o_ref| over the head's checked rows;
@@ -100,13 +104,27 @@ def compare_vs(h, sel_v_gpu, sel_s_gpu, idx, alpha, rep: Report):
     rep.vs_flips[h] = flips
 
 
-def compare_pe(h, mask_gpu, idx, rep: Report):
+def _mass_before(pe, nb):
+    """Cumulative mass of the entries ranked before each causal entry in the
+    oracle's order (value descending, flat index ascending), as [nb, nb]."""
+    r, c = np.tril_indices(nb)
+    a = pe.values[r, c]
+    order = np.lexsort((r * nb + c, -a))
+    before = np.empty(len(a))
+    before[order] = np.concatenate(([0.0], np.cumsum(a[order])[:-1]))
+    out = np.zeros((nb, nb))
+    out[r, c] = before
+    return out
+
+
+def compare_pe(h, mask_gpu, idx, rep: Report, gamma: float = None):
     pe = idx.pe
     nb = pe.mask.shape[0]
     gpu = mask_gpu[:nb, :nb]
     bad = np.argwhere(gpu != pe.mask)
     flips = 0
     cut = pe.cut_value
+    before = None
     for r, c in bad:
         if c > r:
             rep.failures.append(f"head {h}: PE mask set above the diagonal at ({r},{c})")
@@ -114,9 +132,15 @@ def compare_pe(h, mask_gpu, idx, rep: Report):
         v = pe.values[r, c]
         if cut > 0 and abs(v - cut) <= REL_FLIP * cut:
             flips += 1
-        else:
-            rep.failures.append(f"head {h}: PE block ({r},{c}) gpu={gpu[r, c]} oracle={pe.mask[r, c]} "
-                                f"value={v:.6g} cut={cut:.6g}")
+            continue
+        if gamma is not None and gamma < 1.0:
+            if before is None:
+                before = _mass_before(pe, nb)
+            if abs(before[r, c] - gamma) <= REL_FLIP * gamma:
+                flips += 1
+                continue
+        rep.failures.append(f"head {h}: PE block ({r},{c}) gpu={gpu[r, c]} oracle={pe.mask[r, c]} "
+                            f"value={v:.6g} cut={cut:.6g}")
     rep.pe_flips[h] = flips
 
 

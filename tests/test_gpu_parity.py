@@ -95,7 +95,7 @@ def check_index(host, oidx, cfg, rep):
         assert (host["v_idx"][h][:nv] == np.nonzero(host["sel_v"][h])[0]).all()
         assert (host["s_idx"][h][:ns] == np.nonzero(host["sel_s"][h])[0]).all()
         if idx.route == O.PE and int(host["route"][h]) == O.PE:
-            P.compare_pe(h, host["pe"][h], idx, rep)
+            P.compare_pe(h, host["pe"][h], idx, rep, f32(cfg.gamma))
             assert int(host["pe_count"][h]) == int(host["pe"][h][np.tril_indices(cfg.n_blocks)].sum())
         # the block masses themselves (float32 device sums vs float64)
         np.testing.assert_allclose(host["p_v"][h], idx.p_v, rtol=2e-3, atol=2e-6)

@@ -69,3 +69,26 @@ def test_flip_bound_is_per_head_and_per_kind():
         pass
     else:
         raise AssertionError("2 of 128 VS flips exceeds 1%")
+
+
+def test_pe_block_on_the_gamma_threshold_is_a_flip():
+    # a 3x3 causal map already normalised: sorted 0.4 (0,0), 0.2 (2,0), 0.15 (2,1),
+    # 0.1 (1,0), 0.1 (1,1), 0.05 (2,2); gamma = 0.6 is reached by the first two,
+    # so (2,1) sits on the threshold (mass before it = gamma) while (1,0) does not
+    vals = np.array([[0.4, 0.0, 0.0], [0.1, 0.1, 0.0], [0.2, 0.15, 0.05]])
+    sel = O.gamma_select(vals, 0.6)
+    assert sel.k_star == 2
+    idx = O.HeadIndex(0.0, O.PE, None, None, None, None, 0.0, 0.0, sel)
+    gpu = sel.mask.copy()
+    gpu[2, 1] = True                  # value 0.15, 25% from the cut 0.2
+    rep = P.Report()
+    P.compare_pe(0, gpu, idx, rep)    # by value alone: a failure
+    assert rep.failures
+    rep = P.Report()
+    P.compare_pe(0, gpu, idx, rep, 0.6)
+    assert not rep.failures and rep.pe_flips[0] == 1
+    gpu2 = sel.mask.copy()
+    gpu2[1, 0] = True                 # mass before it is 0.75: far from gamma
+    rep = P.Report()
+    P.compare_pe(0, gpu2, idx, rep, 0.6)
+    assert rep.failures
