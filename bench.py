@@ -665,8 +665,9 @@ def run_stage(args):
     import torch
     import long_context_prefill_last_b200 as crisp
     c = S.CONFIGS[args.config]
-    if args.n or args.h_q or args.h_kv:
-        c = S.scaled(args.config, n=args.n, h_q=args.h_q, h_kv=args.h_kv)
+    if args.n or args.h_q or args.h_kv or args.planted is not None:
+        pg = None if args.planted is None else [int(x) for x in args.planted.split(",") if x.strip()]
+        c = S.scaled(args.config, n=args.n, h_q=args.h_q, h_kv=args.h_kv, planted_groups=pg)
     layer = S.generate(c, threads=min(32, os.cpu_count() or 8))
     q, k, v = (t.cuda() for t in S.to_torch(layer))
     out = torch.empty_like(q)
@@ -734,6 +735,8 @@ def parse_args(argv=None):
     ap.add_argument("--n", type=int, help="profiling mode: scaled sequence length")
     ap.add_argument("--h-q", type=int, help="profiling mode: scaled query heads")
     ap.add_argument("--h-kv", type=int, help="profiling mode: scaled KV heads")
+    ap.add_argument("--planted", help="profiling mode: comma-separated planted KV groups of the scaled layer "
+                                      "('' for none: every group Gaussian)")
     return ap.parse_args(argv)
 
 

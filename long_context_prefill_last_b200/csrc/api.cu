@@ -39,6 +39,7 @@ WsLayout ws_layout(const Shape& s) {
   L.row_stat = take(hq * nb * 8);
   L.tile_kr = take(hq * (size_t)s.nt * s.nt * 4 * 8);
   L.tie_cnt = take(hq * nb * (size_t)s.nt * 4);
+  L.tie_row = take(hq * nb * 4);
   L.hist = take(hq * sizeof(PeHist));
   L.pe_state = take(hq * sizeof(PeState));
   L.kv_pe = take(hkv * 4);

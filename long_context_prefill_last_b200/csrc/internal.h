@@ -30,7 +30,8 @@ struct WsLayout {
   size_t khi, klo;    // bf16 [h_kv][nt*128][d]      pooled K, hi and lo parts (rows past N_b zero)
   size_t row_stat;    // f32x2 [h_q][N_b]            pooled-map row (maximum, 1 / (sum * N_b)), log2 domain
   size_t tile_kr;     // u32x2 [h_q][nt][nt][4]      (min, max) key of each 32-row quarter of a 128x128 map tile
-  size_t tie_cnt;     // u32 [h_q][N_b][nt]          entries equal to the cut per (row, tile), then offsets
+  size_t tie_cnt;     // u32 [h_q][N_b][nt]          entries equal to the cut in the row before each tile
+  size_t tie_row;     // u32 [h_q][N_b]              entries equal to the cut per row, then offsets
   size_t hist;        // per head: PeHist
   size_t pe_state;    // per head: PeState
   size_t kv_pe;       // int32 [h_kv]: 1 if any query head of the group routes PE
@@ -75,9 +76,13 @@ struct IndexPtrs {
 constexpr int kHistL0 = 4096;   // bits 31..20
 constexpr int kHistL1 = 4096;   // bits 19..8
 constexpr int kHistL2 = 256;    // bits 7..0
+// Mass is kept in fixed point, units of 2^-62 (every entry of the normalised
+// map is at most 1/4, the total is 1): integer sums are exact in any order,
+// so the cut does not depend on the order of the atomics.
+constexpr double kMassUnit = 1.0 / 4611686018427387904.0;   // 2^-62
 struct PeHist {
   unsigned long long count[kHistL0];
-  double mass[kHistL0];
+  unsigned long long mass[kHistL0];
 };
 struct PeState {
   double s_above;       // mass strictly above the current key prefix

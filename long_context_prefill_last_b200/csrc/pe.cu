@@ -21,9 +21,10 @@
 //      smallest and largest key;
 //   2. level 1 (bits 19..8) and level 2 (bits 7..0): only tiles whose key
 //      range meets the prefix found so far are recomputed;
-//   3. ties (only when the cut keeps part of the entries equal to it): per
-//      (row, tile) counts of entries equal to the cut, then a scan in flat
-//      order;
+//   3. ties (only when the cut keeps part of the entries equal to it): one
+//      warpgroup walks each stripe, so every row's count of entries equal to
+//      the cut builds up in a register (its value before each tile is kept),
+//      then the row totals are scanned in flat order;
 //   4. masks: tiles entirely above (below) the cut are written without
 //      recomputation; the rest are recomputed and compared.
 #include <cuda.h>
@@ -49,7 +50,8 @@ struct PeArgs {
   const __nv_bfloat16* qlo;   // [h_q][nb][128]  bf16(Q-bar * scale_log2 - qhi)
   float2* row_stat;           // [h_q][nb]        (row maximum, 1 / (row sum * N_b)), log2 domain
   uint2* tile_kr;             // [h_q][nt][nt][4] (min key, max key) per 32-row quarter of a tile
-  uint32_t* tie_cnt;          // [h_q][nb][nt]    ties per (row, tile), then exclusive offsets
+  uint32_t* tie_cnt;          // [h_q][nb][nt]    ties of the row in the tiles before each tile
+  uint32_t* tie_row;          // [h_q][nb]        ties per row, then exclusive offsets in flat order
   PeHist* hist;
   PeState* state;
   uint32_t* pe_mask;
@@ -113,12 +115,17 @@ __global__ void __launch_bounds__(kPoolThreads) pe_pool_kernel(const T* __restri
   // past N_b are written as zeros so its TMA boxes never leave the tensor)
   const long long q_items = (long long)h_q * nb;
   const long long items = q_items + (long long)h_kv * nb_pad;
-  for (long long it = blockIdx.x; it < items; it += gridDim.x) {
+  const long long G = gridDim.x;
+  for (long long it = blockIdx.x; it < items; it += G) {
     const bool is_q = it < q_items;
     const int hh = is_q ? (int)(it / nb) : (int)((it - q_items) / nb_pad);
     const int b = is_q ? (int)(it % nb) : (int)((it - q_items) % nb_pad);
     const bool want = is_q ? route[hh] == 1 : kv_pe[hh] != 0;
-    if (!want) continue;   // uniform over the CTA
+    if (!want) {   // uniform over the CTA: jump to this CTA's first item of the next head
+      const long long next = is_q ? (long long)(hh + 1) * nb : q_items + (long long)(hh + 1) * nb_pad;
+      it += ((next - it + G - 1) / G - 1) * G;
+      continue;
+    }
     float acc[N];
 #pragma unroll
     for (int j = 0; j < N; ++j) acc[j] = 0.f;
@@ -168,7 +175,7 @@ constexpr uint32_t kHalfBytes = 128 * 128;
 constexpr int kHistMax = kHistL1;                // largest per-CTA histogram (level 1)
 constexpr uint32_t OFF_K = 0;                                      // [stage][hi, lo] K-bar tiles
 constexpr uint32_t OFF_HCNT = OFF_K + kStages * 2 * kTileBytes;    // u32 [kHistMax]
-constexpr uint32_t OFF_HMASS = OFF_HCNT + kHistMax * 4;            // f64 [kHistMax]
+constexpr uint32_t OFF_HMASS = OFF_HCNT + kHistMax * 4;            // u64 [kHistMax], fixed-point mass
 constexpr uint32_t OFF_XCH = OFF_HMASS + kHistMax * 8;             // float2 [128]: row statistics exchange
 constexpr uint32_t OFF_ROW = OFF_XCH + 128 * 8;                    // float2 [128]: (m, inv) of the stripe's rows
 constexpr uint32_t OFF_BAR = OFF_ROW + 128 * 8;
@@ -310,9 +317,24 @@ __device__ __forceinline__ bool epi_sync(uint32_t sbase, uint32_t& phase, volati
   return ok;
 }
 
-__device__ __forceinline__ void hist_add(uint32_t* cnt, double* mass, uint32_t b, uint32_t c, double m) {
+// An entry's mass in fixed point (units of 2^-62; entries are at most 1/4).
+__device__ __forceinline__ unsigned long long mass_fixed(float v) { return __float2ull_rn(v * 0x1p62f); }
+
+__device__ __forceinline__ void hist_add(uint32_t* cnt, unsigned long long* mass, uint32_t b, uint32_t c,
+                                         unsigned long long m) {
   atomicAdd(&cnt[b], c);
   atomicAdd(&mass[b], m);
+}
+
+__device__ __forceinline__ uint32_t warp_sum_u32(uint32_t v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ unsigned long long warp_sum_u64(unsigned long long v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
 }
 
 template <int MODE>
@@ -325,7 +347,7 @@ pe_sweep_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sgen + OFF_ABORT);
   uint32_t* tmem_ptr_smem = reinterpret_cast<uint32_t*>(sgen + OFF_TMEMPTR);
   uint32_t* hcnt = reinterpret_cast<uint32_t*>(sgen + OFF_HCNT);
-  double* hmass = reinterpret_cast<double*>(sgen + OFF_HMASS);
+  unsigned long long* hmass = reinterpret_cast<unsigned long long*>(sgen + OFF_HMASS);
   float2* xch = reinterpret_cast<float2*>(sgen + OFF_XCH);
   float2* rows_sm = reinterpret_cast<float2*>(sgen + OFF_ROW);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -349,7 +371,7 @@ pe_sweep_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
   }
   for (int i = threadIdx.x; i < kHistMax; i += kThreads) {
     hcnt[i] = 0u;
-    hmass[i] = 0.0;
+    hmass[i] = 0ull;
   }
   __syncthreads();
   if (*abort_flag) return;   // an earlier kernel failed: do nothing (uniform, before TMEM is taken)
@@ -512,15 +534,21 @@ pe_sweep_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
         if (head_live(a, MODE, hn, cn) && stripe_mask(a, cn, hn, rtn, lane) != 0) return true;
       return false;
     };
-    // one S tile into registers (and the buffer released)
-    auto load_s = [&](float (&s)[128]) -> bool {
+    // Quarter q (columns [32q, 32q + 32)) of the S tile j into x; the first
+    // quarter waits for the tile, the last releases its buffer once loaded.
+    auto load_q = [&](int qq, float (&x)[32]) -> bool {
       const int buf = j & 1;
-      if (!warp_wait(bar_addr(sbase, B_SFULL + buf), (j >> 1) & 1, abort_flag, a.status, 46)) return false;
-      dev::tc_fence_after();
-      dev::tmem_ld128(tmem + lane_base + (uint32_t)buf * 128u, s);
+      if (qq == 0) {
+        if (!warp_wait(bar_addr(sbase, B_SFULL + buf), (j >> 1) & 1, abort_flag, a.status, 46)) return false;
+        dev::tc_fence_after();
+      }
+      dev::tmem_ld32(tmem + lane_base + (uint32_t)buf * 128u + (uint32_t)qq * 32u,
+                     reinterpret_cast<uint32_t (&)[32]>(x));
       dev::tmem_wait_ld();
-      dev::tc_fence_before();
-      dev::mbar_arrive(bar_addr(sbase, B_SEMPTY + buf));
+      if (qq == 3) {
+        dev::tc_fence_before();
+        dev::mbar_arrive(bar_addr(sbase, B_SEMPTY + buf));
+      }
       return true;
     };
     auto flush_hist = [&](int hh) -> bool {
@@ -532,7 +560,7 @@ pe_sweep_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
           atomicAdd(&gh->count[i], (unsigned long long)cnt);
           atomicAdd(&gh->mass[i], hmass[i]);
           hcnt[i] = 0u;
-          hmass[i] = 0.0;
+          hmass[i] = 0ull;
         }
       }
       return epi_sync(sbase, epi_phase, abort_flag, a.status);
@@ -542,8 +570,10 @@ pe_sweep_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
       int h0, rt0;
       if (next_active(-1, h0, rt0)) ok = write_q(h0, rt0, 0);
     }
+    int li = -1;   // live stripes so far
     for (int it = 0; ok && item_of(a, blockIdx.x, it, h, rt); ++it) {
       if (!head_live(a, MODE, h, c)) continue;
+      ++li;
       const uint64_t act_mask = stripe_mask(a, c, h, rt, lane);
       const uint64_t above_mask = (MODE == kMask && !c.all) ? stripe_above(a, c, h, rt, lane) : 0ull;
       const int n_act = __popcll(act_mask);
@@ -560,28 +590,32 @@ pe_sweep_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
       // last valid column of tile ct: every column before the diagonal tile
       // (c <= r < N_b), up to the diagonal in it, none in a padding row
       auto last_of = [&](int ct) { return !row_ok ? -1 : (ct < rt ? 127 : ncol); };
-      float s[128];
+      float x[32];
       if (MODE == kStatsHist0) {
-        // sweep 1: this warpgroup's tiles, online maximum and normaliser per row
+        // sweep 1: this warpgroup's tiles, running maximum and normaliser per row
         float m = -INFINITY, l = 0.f;
         for (int ct = 0; ct <= rt; ++ct, ++j) {
           if ((j & 1) != wg) continue;
-          if (!load_s(s)) {
-            ok = false;
-            break;
-          }
           const int last = last_of(ct);
-          float tmax = -INFINITY;
+#pragma unroll 1
+          for (int qq = 0; qq < 4; ++qq) {
+            if (!load_q(qq, x)) {
+              ok = false;
+              break;
+            }
+            const int lastc = last - 32 * qq;   // valid: i <= lastc
+            float hm = -INFINITY;
 #pragma unroll
-          for (int cc = 0; cc < 128; ++cc) tmax = cc <= last ? fmaxf(tmax, s[cc]) : tmax;
-          if (tmax > m) {
-            l *= dev::ex2(m - tmax);
-            m = tmax;
+            for (int i = 0; i < 32; ++i) hm = i <= lastc ? fmaxf(hm, x[i]) : hm;
+            const float mn = fmaxf(m, hm);
+            l *= mn == m ? 1.f : dev::ex2(m - mn);
+            m = mn;
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int i = 0; i < 32; ++i) acc[i & 3] += dev::ex2(i <= lastc ? x[i] - m : -INFINITY);
+            l += (acc[0] + acc[1]) + (acc[2] + acc[3]);
           }
-          float sum = 0.f;
-#pragma unroll
-          for (int cc = 0; cc < 128; ++cc) sum += cc <= last ? dev::ex2(s[cc] - m) : 0.f;
-          l += sum;
+          if (!ok) break;
         }
         if (!ok) break;
         // the two warpgroups' statistics of each row, combined
@@ -603,34 +637,68 @@ pe_sweep_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
           break;
         }
         const float2 st = rows_sm[lr];
-        // sweep 2: entries, level-0 histogram (runs of equal buckets merged), tile key ranges
+        // A row's largest entry is its normaliser inv (at l = m), so its
+        // entries fall in level-0 buckets at or below that of inv; the rows
+        // of a warp sit close together. Counts and mass of the four buckets
+        // below the warp's highest are kept in registers (predicated adds)
+        // and summed over the warp once per tile; the rare entries further
+        // down go to the shared histogram one by one.
+        const uint32_t b_row = row_ok ? (__float_as_uint(st.y) >> 20) : 0u;
+        uint32_t b_base = b_row;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) b_base = max(b_base, __shfl_xor_sync(0xffffffffu, b_base, o));
+        // sweep 2: entries, level-0 histogram, tile key ranges
         for (int ct = 0; ct <= rt; ++ct, ++j) {
           if ((j & 1) != wg) continue;
-          if (!load_s(s)) {
-            ok = false;
-            break;
-          }
           const int last = last_of(ct);
-          uint32_t kmin = 0xFFFFFFFFu, kmax = 0u, cur = 0xFFFFFFFFu, cnt = 0u;
-          double mass = 0.0;
-#pragma unroll
-          for (int cc = 0; cc < 128; ++cc) {
-            if (cc > last) continue;
-            const float v = entry_value(s[cc], st.x, st.y);
-            const uint32_t key = __float_as_uint(v);
-            kmin = min(kmin, key);
-            kmax = max(kmax, key);
-            const uint32_t b = key >> 20;
-            if (b != cur) {
-              if (cnt) hist_add(hcnt, hmass, cur, cnt, mass);
-              cur = b;
-              cnt = 0u;
-              mass = 0.0;
+          uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+          uint32_t c0 = 0, c1 = 0, c2 = 0, c3 = 0;
+          unsigned long long m0 = 0, m1 = 0, m2 = 0, m3 = 0;
+#pragma unroll 1
+          for (int qq = 0; qq < 4; ++qq) {
+            if (!load_q(qq, x)) {
+              ok = false;
+              break;
             }
-            ++cnt;
-            mass += (double)v;
+            const int lastc = last - 32 * qq;
+            bool far = false;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const bool valid = i <= lastc;
+              const float v = dev::ex2(valid ? x[i] - st.x : -INFINITY) * st.y;
+              const uint32_t key = __float_as_uint(v);
+              kmin = valid ? min(kmin, key) : kmin;
+              kmax = valid ? max(kmax, key) : kmax;
+              const uint32_t off = valid ? b_base - (key >> 20) : 0xFFFFFFFFu;
+              const unsigned long long fx = mass_fixed(v);
+              c0 += off == 0 ? 1u : 0u;
+              m0 += off == 0 ? fx : 0ull;
+              c1 += off == 1 ? 1u : 0u;
+              m1 += off == 1 ? fx : 0ull;
+              c2 += off == 2 ? 1u : 0u;
+              m2 += off == 2 ? fx : 0ull;
+              c3 += off == 3 ? 1u : 0u;
+              m3 += off == 3 ? fx : 0ull;
+              far = far || (valid && off > 3u);
+            }
+            if (__any_sync(0xffffffffu, far)) {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                const bool valid = i <= lastc;
+                const float v = dev::ex2(valid ? x[i] - st.x : -INFINITY) * st.y;
+                const uint32_t key = __float_as_uint(v);
+                if (valid && b_base - (key >> 20) > 3u) hist_add(hcnt, hmass, key >> 20, 1u, mass_fixed(v));
+              }
+            }
           }
-          if (cnt) hist_add(hcnt, hmass, cur, cnt, mass);
+          if (!ok) break;
+          const uint32_t cs[4] = {warp_sum_u32(c0), warp_sum_u32(c1), warp_sum_u32(c2), warp_sum_u32(c3)};
+          const unsigned long long ms[4] = {warp_sum_u64(m0), warp_sum_u64(m1), warp_sum_u64(m2), warp_sum_u64(m3)};
+          if (lane == 0) {
+#pragma unroll
+            for (int w = 0; w < 4; ++w)
+              if (cs[w] && b_base >= (uint32_t)w) hist_add(hcnt, hmass, b_base - w, cs[w], ms[w]);
+          }
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) {
             kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
@@ -648,7 +716,41 @@ pe_sweep_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
         uint32_t* mrow = a.pe_mask + ((size_t)h * a.nb + (row_ok ? r : 0)) * a.words;
         uint32_t* trow = a.tie_cnt + ((size_t)h * a.nb + (row_ok ? r : 0)) * a.nt;
         unsigned long long kept = 0;
-        for (int ct = 0; ct <= rt; ++ct) {
+        if (MODE == kTies) {
+          // warpgroup li % 2 takes every tile of this stripe, so each row's
+          // count of entries equal to the cut builds up in one register
+          const bool mine = (li & 1) == wg;
+          uint32_t run = 0;
+          for (int ct = 0; ct <= rt; ++ct) {
+            const bool act = (act_mask >> ct) & 1ull;
+            if (!mine) {
+              if (act) ++j;
+              continue;
+            }
+            if (row_ok) trow[ct] = run;
+            if (!act) continue;
+            const int last = last_of(ct);
+#pragma unroll 1
+            for (int qq = 0; qq < 4; ++qq) {
+              if (!load_q(qq, x)) {
+                ok = false;
+                break;
+              }
+              const int lastc = last - 32 * qq;
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                const bool valid = i <= lastc;
+                const uint32_t key = __float_as_uint(dev::ex2(valid ? x[i] - st.x : -INFINITY) * st.y);
+                run += (valid && key == c.cut) ? 1u : 0u;
+              }
+            }
+            if (!ok) break;
+            ++j;
+          }
+          if (!ok) break;
+          if (mine && row_ok) a.tie_row[(size_t)h * a.nb + r] = run;
+        }
+        for (int ct = 0; MODE != kTies && ct <= rt; ++ct) {
           const bool act = (act_mask >> ct) & 1ull;
           const int last = last_of(ct);
           const int owner = act ? (j & 1) : (ct & 1);
@@ -656,62 +758,73 @@ pe_sweep_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
             if (act) ++j;
             continue;
           }
-          if (act) {
-            if (!load_s(s)) {
-              ok = false;
-              break;
-            }
-            ++j;
-          }
           if (MODE == kHist1 || MODE == kHist2) {
             const int shift_p = MODE == kHist1 ? 20 : 8;
             const int shift_b = MODE == kHist1 ? 8 : 0;
             const uint32_t bmask = MODE == kHist1 ? 0xFFFu : 0xFFu;
+#pragma unroll 1
+            for (int qq = 0; qq < 4; ++qq) {
+              if (!load_q(qq, x)) {
+                ok = false;
+                break;
+              }
+              const int lastc = last - 32 * qq;
 #pragma unroll
-            for (int cc = 0; cc < 128; ++cc) {
-              if (cc > last) continue;
-              const float v = entry_value(s[cc], st.x, st.y);
-              const uint32_t key = __float_as_uint(v);
-              if ((key >> shift_p) == c.prefix) hist_add(hcnt, hmass, (key >> shift_b) & bmask, 1u, (double)v);
-            }
-          } else if (MODE == kTies) {
-            uint32_t ties = 0;
-            if (act) {
-#pragma unroll
-              for (int cc = 0; cc < 128; ++cc) {
-                if (cc > last) continue;
-                ties += __float_as_uint(entry_value(s[cc], st.x, st.y)) == c.cut ? 1u : 0u;
+              for (int i = 0; i < 32; ++i) {
+                const bool valid = i <= lastc;
+                const float v = dev::ex2(valid ? x[i] - st.x : -INFINITY) * st.y;
+                const uint32_t key = __float_as_uint(v);
+                if (valid && (key >> shift_p) == c.prefix)
+                  hist_add(hcnt, hmass, (key >> shift_b) & bmask, 1u, mass_fixed(v));
               }
             }
-            if (row_ok) trow[ct] = ties;
+            if (!ok) break;
+            ++j;
           } else {   // kMask
             uint32_t w[4] = {0u, 0u, 0u, 0u};
-            if (row_ok) {
-              if (c.all || ((above_mask >> ct) & 1ull)) {   // every entry kept
+            if (c.all || ((above_mask >> ct) & 1ull)) {   // every entry kept
 #pragma unroll
-                for (int cc = 0; cc < 128; ++cc)
-                  if (cc <= last) w[cc >> 5] |= 1u << (cc & 31);
-              } else if (act) {
-                unsigned long long rank = c.partial_ties ? trow[ct] : 0ull;
-#pragma unroll
-                for (int cc = 0; cc < 128; ++cc) {
-                  if (cc > last) continue;
-                  const uint32_t key = __float_as_uint(entry_value(s[cc], st.x, st.y));
-                  bool keep = key > c.cut || (ct == rt && cc == last);
-                  if (key == c.cut) {
-                    keep = keep || !c.partial_ties || rank < c.t_keep;
-                    ++rank;
-                  }
-                  if (keep) w[cc >> 5] |= 1u << (cc & 31);
+              for (int cc = 0; cc < 128; ++cc)
+                if (cc <= last) w[cc >> 5] |= 1u << (cc & 31);
+            } else if (act) {
+              unsigned long long rank =
+                  c.partial_ties && row_ok ? (unsigned long long)a.tie_row[(size_t)h * a.nb + r] + trow[ct] : 0ull;
+              const int diag = ct == rt ? ncol : -1;
+#pragma unroll 1
+              for (int qq = 0; qq < 4; ++qq) {
+                if (!load_q(qq, x)) {
+                  ok = false;
+                  break;
                 }
+                const int lastc = last - 32 * qq;
+                uint32_t word = 0u;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                  const bool valid = i <= lastc;
+                  const uint32_t key = __float_as_uint(dev::ex2(valid ? x[i] - st.x : -INFINITY) * st.y);
+                  const bool tie = valid && key == c.cut;
+                  const bool keep = (valid && key > c.cut) || (tie && (!c.partial_ties || rank < c.t_keep)) ||
+                                    (32 * qq + i == diag);
+                  rank += tie ? 1ull : 0ull;
+                  word |= keep ? 1u << i : 0u;
+                }
+                // w[qq] with qq a loop variable would live in local memory: select instead
+                w[0] = qq == 0 ? word : w[0];
+                w[1] = qq == 1 ? word : w[1];
+                w[2] = qq == 2 ? word : w[2];
+                w[3] = qq == 3 ? word : w[3];
               }
+              if (!ok) break;
+              ++j;
+            }
+            if (row_ok) {
               if (ct == rt) w[ncol >> 5] |= 1u << (ncol & 31);   // the diagonal block
 #pragma unroll
-              for (int x = 0; x < 4; ++x) {
-                const int word = ct * 4 + x;
+              for (int x4 = 0; x4 < 4; ++x4) {
+                const int word = ct * 4 + x4;
                 if (word < a.words) {
-                  mrow[word] = w[x];
-                  kept += __popc(w[x]);
+                  mrow[word] = w[x4];
+                  kept += __popc(w[x4]);
                 }
               }
             }
@@ -779,7 +892,7 @@ __global__ void __launch_bounds__(1024) pe_find_kernel(PeArgs a, int level) {
   double my = 0.0;
   for (int u = 0; u < per; ++u) {
     const int b = nbk - 1 - (tid * per + u);
-    if (b >= 0) my += hist->mass[b];
+    if (b >= 0) my += (double)hist->mass[b] * kMassUnit;
   }
   tsum[tid] = my;
   __syncthreads();
@@ -806,7 +919,7 @@ __global__ void __launch_bounds__(1024) pe_find_kernel(PeArgs a, int level) {
         if (hist->count[b] == 0) continue;
         last_b = b;
         last_above = acc;
-        const double nxt = acc + hist->mass[b];
+        const double nxt = acc + (double)hist->mass[b] * kMassUnit;
         if (nxt >= gamma) break;
         acc = nxt;
       }
@@ -824,7 +937,7 @@ __global__ void __launch_bounds__(1024) pe_find_kernel(PeArgs a, int level) {
     for (int b = 0; b < nbk; ++b) {
       if (hist->count[b] > 0) {
         s_bucket = b;
-        s_above_new = base + (tsum[1023] - hist->mass[b]);
+        s_above_new = base + (tsum[1023] - (double)hist->mass[b] * kMassUnit);
         s_found = 1;
         break;
       }
@@ -856,26 +969,25 @@ __global__ void __launch_bounds__(1024) pe_find_kernel(PeArgs a, int level) {
   __syncthreads();
   for (int b = tid; b < kHistL0; b += 1024) {
     hist->count[b] = 0;
-    hist->mass[b] = 0.0;
+    hist->mass[b] = 0ull;
   }
 }
 
-// Exclusive scan, in flat order (row by row, tiles left to right), of the
-// per-(row, tile) tie counts of heads whose cut keeps part of its ties.
-// One CTA of 1024 threads per head; entries (r, ct) with ct > r / 128 hold
-// nothing and are not read.
+// Exclusive scan over rows of the per-row tie counts, for heads whose cut
+// keeps part of its ties: flat order is row by row, so a tie's rank is its
+// row's offset plus the ties before it in the row (kept per tile by the
+// ties pass). One CTA of 1024 threads per head.
 __global__ void __launch_bounds__(1024) pe_tie_scan_kernel(PeArgs a) {
   const int h = blockIdx.x;
   if (a.route[h] != 1) return;
   const PeState* st = a.state + h;
   if (st->all || st->t_keep >= st->n_ties) return;
   __shared__ unsigned long long part[1024];
-  uint32_t* cnt = a.tie_cnt + (size_t)h * a.nb * a.nt;
+  uint32_t* rows = a.tie_row + (size_t)h * a.nb;
   const int per = (a.nb + 1023) / 1024;
   const int lo = threadIdx.x * per, hi = min(a.nb, lo + per);
   unsigned long long s = 0;
-  for (int r = lo; r < hi; ++r)
-    for (int ct = 0; ct <= r / 128; ++ct) s += cnt[(size_t)r * a.nt + ct];
+  for (int r = lo; r < hi; ++r) s += rows[r];
   part[threadIdx.x] = s;
   __syncthreads();
   for (int off = 1; off < 1024; off <<= 1) {
@@ -884,15 +996,13 @@ __global__ void __launch_bounds__(1024) pe_tie_scan_kernel(PeArgs a) {
     part[threadIdx.x] += v;
     __syncthreads();
   }
+  // offsets fit 32 bits: a head has at most 2^25 causal blocks
   unsigned long long acc = threadIdx.x > 0 ? part[threadIdx.x - 1] : 0ull;
-  for (int r = lo; r < hi; ++r)
-    for (int ct = 0; ct <= r / 128; ++ct) {
-      uint32_t* e = cnt + (size_t)r * a.nt + ct;
-      const uint32_t v = *e;
-      // offsets beyond 2^32 cannot occur: a head has at most 2^25 causal blocks
-      *e = (uint32_t)acc;
-      acc += v;
-    }
+  for (int r = lo; r < hi; ++r) {
+    const uint32_t v = rows[r];
+    rows[r] = (uint32_t)acc;
+    acc += v;
+  }
 }
 
 template <int MODE>
@@ -925,6 +1035,7 @@ cudaError_t launch_pe(const void* q, const void* k, const Shape& s, char* ws, co
   a.row_stat = reinterpret_cast<float2*>(ws + L.row_stat);
   a.tile_kr = reinterpret_cast<uint2*>(ws + L.tile_kr);
   a.tie_cnt = reinterpret_cast<uint32_t*>(ws + L.tie_cnt);
+  a.tie_row = reinterpret_cast<uint32_t*>(ws + L.tie_row);
   a.hist = reinterpret_cast<PeHist*>(ws + L.hist);
   a.state = reinterpret_cast<PeState*>(ws + L.pe_state);
   a.pe_mask = ix.pe_mask;

@@ -7,8 +7,10 @@
 // CTA and used for two 128-row M tiles (four query heads).
 //
 // CTA = (KV head, pair of M tiles, contiguous range of 8-tile chunks);
-// 10 warps: 0 TMA producer, 1 TMEM + MMA issuer, 2..9 softmax (one row per
-// thread; warps 2..5 take M tile 0, 6..9 M tile 1).
+// 12 warps: 0 TMA producer, 1 TMEM + MMA issuer, 2..3 idle, 4..11 softmax (one
+// row per thread; warps 4..7 take M tile 0, 8..11 M tile 1). The first
+// warpgroup gives registers to the softmax warpgroups (setmaxnreg 64 / 216 /
+// 216), which hold a 128-column row and the chunk's 16 partial sums.
 // TMEM: S[m][buf] at columns (2m + buf) * 128, 512 columns in all.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -21,18 +23,22 @@
 namespace crisp {
 namespace {
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;
+constexpr int kRegsControl = 64;
+constexpr int kRegsSoftmax = 216;
+static_assert(128 * kRegsControl + 256 * kRegsSoftmax <= kThreads * 168, "register split exceeds the launch");
 constexpr int kStages = 4;
 // Pairs in every 8 whose exponentials use the FMA-pipe polynomial instead of
-// MUFU. The proxy's softmax is not MUFU-bound at d = 128 (the per-row issue
-// of the max, scale and sums dominates), so all exponentials stay on MUFU.
-constexpr int kPolyPairsPer8 = 0;
+// MUFU. With the chunk partials in registers the softmax is led by MUFU, and
+// moving one pair in eight to the polynomial measured 8% faster on the route
+// stage at 512K tokens (two in eight: 4% faster, the extra FMA-pipe
+// instructions then cost more than the MUFU time they free).
+constexpr int kPolyPairsPer8 = 1;
 constexpr uint32_t kTileBytes = 128 * 128 * 2;
 constexpr uint32_t kHalfBytes = 128 * 128;
 constexpr uint32_t OFF_Q = 0;                                // 2 M tiles
 constexpr uint32_t OFF_K = OFF_Q + 2 * kTileBytes;
-constexpr uint32_t OFF_PART = OFF_K + kStages * kTileBytes;   // [2*kChunkTiles][256] f32
-constexpr uint32_t OFF_BAR = OFF_PART + 2 * kChunkTiles * 256 * 4;
+constexpr uint32_t OFF_BAR = OFF_K + kStages * kTileBytes;
 enum {
   B_Q = 0,
   B_KFULL = 1,
@@ -121,6 +127,7 @@ proxy_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   const uint32_t tmem = *tmem_ptr_smem;
   const int n_mt = heads_here > 2 ? 2 : 1;   // M tiles holding at least one head
 
+  if (warp < 4) dev::regs_release<kRegsControl>();
   if (warp == 0) {
     if (lane == 0) {
       dev::prefetch_tmap(&tm_q);
@@ -183,9 +190,10 @@ proxy_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       dev::umma_commit(bar_addr(sbase, B_DRAIN));
       dev::mbar_drain(bar_addr(sbase, B_DRAIN), 0);
     }
-  } else {
+  } else if (warp >= 4) {
     // ---------------------------------------------------------------- softmax warps
-    const int sw = warp - 2;                 // 0..7
+    dev::regs_acquire<kRegsSoftmax>();
+    const int sw = warp - 4;                 // 0..7
     const int mt = sw >> 2;                  // M tile
     const int quarter = warp & 3;            // TMEM lane quarter of this warp
     const int r = quarter * 32 + lane;       // row inside the M tile
@@ -197,8 +205,11 @@ proxy_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const float sl2 = a.scale_log2;
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const size_t row = (size_t)(head0 + (active ? j : 0)) * kProxyRows + ri;
-    // this thread's chunk partials: part[(2u + {0 lo, 1 hi}) * 256 + sw*32 + lane]
-    float* part = reinterpret_cast<float*>(sgen + OFF_PART) + sw * 32 + lane;
+    // this thread's partials of the current 8-tile chunk, in registers (slot u
+    // of tile t_begin + 8c + u; every slot index below is a compile-time constant)
+    float plo[kChunkTiles], phi[kChunkTiles];
+#pragma unroll
+    for (int w = 0; w < kChunkTiles; ++w) plo[w] = phi[w] = 0.f;
     int k = 0;
     bool ok = true;
     float m_run = -INFINITY, l_run = 0.f;
@@ -232,12 +243,13 @@ proxy_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           mx[3] = dev::max3(mx[3], x[c + 6], x[c + 7]);
         }
         const float tmax = fmaxf(dev::max3(mx[0], mx[1], mx[2]), mx[3]) * sl2;
-        if (tmax > m_run + 8.f) {   // lazy rescale of this chunk's partials
+        if (tmax > m_run + 8.f) {   // lazy rescale of this chunk's partials (slots >= u are still 0)
           const float f = dev::ex2(m_run - tmax);
           l_run *= f;
-          for (int w = 0; w < u; ++w) {
-            part[(2 * w) * 256] *= f;
-            part[(2 * w + 1) * 256] *= f;
+#pragma unroll
+          for (int w = 0; w < kChunkTiles; ++w) {
+            plo[w] *= f;
+            phi[w] *= f;
           }
           m_run = tmax;
         }
@@ -274,20 +286,34 @@ proxy_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const float stot = ((t8[0] + t8[1]) + (t8[2] + t8[3])) + ((t8[4] + t8[5]) + (t8[6] + t8[7]));
         const float shi = (h4[0] + h4[1]) + (h4[2] + h4[3]);
         const float slo = stot - shi;
-        part[(2 * u) * 256] = slo;
-        part[(2 * u + 1) * 256] = shi;
+#pragma unroll
+        for (int w = 0; w < kChunkTiles; ++w) {
+          plo[w] = w == u ? slo : plo[w];
+          phi[w] = w == u ? shi : phi[w];
+        }
         l_run += slo + shi;
         if (u == kChunkTiles - 1 || t == t_end - 1) {
           const int c = t / kChunkTiles;
-          float* plo = a.part_lo + row * a.nb + (size_t)c * kChunkTiles;
-          float* phi = a.part_hi + row * a.nb + (size_t)c * kChunkTiles;
-          for (int w = 0; w <= u; ++w) {
-            plo[w] = part[(2 * w) * 256];
-            phi[w] = part[(2 * w + 1) * 256];
+          float* glo = a.part_lo + row * a.nb + (size_t)c * kChunkTiles;
+          float* ghi = a.part_hi + row * a.nb + (size_t)c * kChunkTiles;
+          if (u == kChunkTiles - 1 && (a.nb & 3) == 0) {   // a whole chunk, 16-byte aligned rows
+            reinterpret_cast<float4*>(glo)[0] = make_float4(plo[0], plo[1], plo[2], plo[3]);
+            reinterpret_cast<float4*>(glo)[1] = make_float4(plo[4], plo[5], plo[6], plo[7]);
+            reinterpret_cast<float4*>(ghi)[0] = make_float4(phi[0], phi[1], phi[2], phi[3]);
+            reinterpret_cast<float4*>(ghi)[1] = make_float4(phi[4], phi[5], phi[6], phi[7]);
+          } else {
+#pragma unroll
+            for (int w = 0; w < kChunkTiles; ++w)
+              if (w <= u) {
+                glo[w] = plo[w];
+                ghi[w] = phi[w];
+              }
           }
           a.chunk_ml[row * a.n_chunks + c] = make_float2(m_run, l_run);
           m_run = -INFINITY;
           l_run = 0.f;
+#pragma unroll
+          for (int w = 0; w < kChunkTiles; ++w) plo[w] = phi[w] = 0.f;
         }
       }
     }
