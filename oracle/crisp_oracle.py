@@ -62,7 +62,7 @@ class OracleCfg:
     w_sink: int = 128         # [S] Eq. (2) text
     w_local: int = 128        # [S] Eq. (2) text
     tau_proxy: float = 0.10   # not given by the pages (our default)
-    alpha: float = 1.0        # [S] Eq. (4) text: calibration-free default
+    alpha: float = 1.0        # [S] Eq. (4): the pages' default multiplier
     gamma: float = 0.95       # PE coverage
     sm_scale: Optional[float] = None   # default 1/sqrt(d)
     force_route: int = -1     # -1 auto, 0 VS, 1 PE
