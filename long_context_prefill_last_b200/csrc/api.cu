@@ -84,7 +84,7 @@ static crisp_status make_shape(const crisp_cfg* c, Shape* s) {
   if (c->dtype != CRISP_BF16 && c->dtype != CRISP_FP32) return CRISP_ERR_DTYPE;
   if (c->d != kHeadDim) return CRISP_ERR_SHAPE;
   if (c->n < 512 || c->n % kBlock != 0 || c->n > (1 << 20)) return CRISP_ERR_SHAPE;
-  if (c->h_q <= 0 || c->h_kv <= 0 || c->h_q % c->h_kv != 0 || c->h_q / c->h_kv > 16 || c->h_q > 1024)
+  if (c->h_q <= 0 || c->h_kv <= 0 || c->h_q % c->h_kv != 0 || c->h_q / c->h_kv > 16 || c->h_q > kMaxHeads)
     return CRISP_ERR_SHAPE;
   if (c->block != kBlock || c->last_q != kProxyRows || c->w_sink != kBlock || c->w_local != kBlock)
     return CRISP_ERR_UNSUPPORTED;

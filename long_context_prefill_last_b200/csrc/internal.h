@@ -72,6 +72,9 @@ struct IndexPtrs {
   float* pe_cut;
 };
 
+// Query heads of one call (after batch folding).
+constexpr int kMaxHeads = 1024;
+
 // Per-head histogram for the PE gamma cut: three radix levels of the fp32 bit pattern.
 constexpr int kHistL0 = 4096;   // bits 31..20
 constexpr int kHistL1 = 4096;   // bits 19..8

@@ -178,7 +178,8 @@ constexpr uint32_t OFF_HCNT = OFF_K + kStages * 2 * kTileBytes;    // u32 [kHist
 constexpr uint32_t OFF_HMASS = OFF_HCNT + kHistMax * 4;            // u64 [kHistMax], fixed-point mass
 constexpr uint32_t OFF_XCH = OFF_HMASS + kHistMax * 8;             // float2 [128]: row statistics exchange
 constexpr uint32_t OFF_ROW = OFF_XCH + 128 * 8;                    // float2 [128]: (m, inv) of the stripe's rows
-constexpr uint32_t OFF_BAR = OFF_ROW + 128 * 8;
+constexpr uint32_t OFF_LIVE = OFF_ROW + 128 * 8;                   // int [kMaxHeads + 1]: count, then PE heads
+constexpr uint32_t OFF_BAR = OFF_LIVE + (((kMaxHeads + 1) * 4 + 7) & ~7);
 enum {
   B_KFULL = 0,
   B_KEMPTY = B_KFULL + kStages,
@@ -213,14 +214,41 @@ __device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile_base, int kk) {
 // every pass evaluates exactly this expression, so they all see the same bits.
 __device__ __forceinline__ float entry_value(float l, float m, float inv) { return dev::ex2(l - m) * inv; }
 
-// Item i of CTA b (snake over items ordered longest stripe first): (head, row tile) or false.
-__device__ __forceinline__ bool item_of(const PeArgs& a, int b, int k, int& h, int& rt) {
-  const int G = gridDim.x;
-  const long long idx = (k & 1) ? (long long)(k + 1) * G - 1 - b : (long long)k * G + b;
-  if (idx >= (long long)a.h_q * a.nt) return false;
-  rt = a.nt - 1 - (int)(idx / a.h_q);
-  h = (int)(idx % a.h_q);
-  return true;
+// Work items. The statistics and tie passes take whole 128-row stripes (their
+// per-row running values need every tile of a row in order); the level-1,
+// level-2 and mask passes split a stripe into segments of kSegTiles tiles,
+// since the tiles they recompute sit in the few stripes whose rows straddle
+// the prefix or the cut, and whole stripes would leave those to a handful of
+// CTAs.
+constexpr int kSegTiles = 8;
+__device__ __forceinline__ bool segmented(int mode) { return mode == kHist1 || mode == kHist2 || mode == kMask; }
+
+struct Item {
+  int h, rt;    // query head, row tile (stripe)
+  int c0, c1;   // tiles c0..c1 of the stripe
+  bool last;    // the segment holding the diagonal tile
+};
+
+// Item k of CTA b: a snake over the items of the heads routed PE (`live`,
+// n_live of them), ordered stripe rt descending, then segment, then head.
+__device__ __forceinline__ bool item_of(const PeArgs& a, const int* live, int n_live, int mode, int b, int k,
+                                        Item& it) {
+  const int G = gridDim.x;   // items per head <= 64 * 8, so every index fits an int
+  int idx = (k & 1) ? (k + 1) * G - 1 - b : k * G + b;
+  for (int rt = a.nt - 1; rt >= 0; --rt) {
+    const int cnt = (segmented(mode) ? rt / kSegTiles + 1 : 1) * n_live;
+    if (idx < cnt) {
+      const int sg = idx / n_live;
+      it.h = live[idx - sg * n_live];
+      it.rt = rt;
+      it.c0 = segmented(mode) ? sg * kSegTiles : 0;
+      it.c1 = segmented(mode) ? min(rt, it.c0 + kSegTiles - 1) : rt;
+      it.last = it.c1 == rt;
+      return true;
+    }
+    idx -= cnt;
+  }
+  return false;
 }
 
 struct PassCtx {
@@ -281,12 +309,12 @@ __device__ __forceinline__ bool tile_active(const PeArgs& a, const PassCtx& c, i
   return kmin <= c.hi_key && kmax >= c.lo_key;
 }
 
-// The tiles ct <= rt of stripe (h, rt) recomputed in this pass, as a bit mask
-// (N_b <= 8192, so at most 64 tiles). Evaluated by a whole warp, one tile per
-// lane, so the key ranges are read in one round.
-__device__ __forceinline__ uint64_t stripe_mask(const PeArgs& a, const PassCtx& c, int h, int rt, int lane) {
-  const bool a0 = lane <= rt && tile_active(a, c, h, rt, lane);
-  const bool a1 = lane + 32 <= rt && tile_active(a, c, h, rt, lane + 32);
+// The tiles c0 <= ct <= c1 of item `it` recomputed in this pass, as a bit
+// mask (N_b <= 8192, so at most 64 tiles). Evaluated by a whole warp, one
+// tile per lane, so the key ranges are read in one round.
+__device__ __forceinline__ uint64_t stripe_mask(const PeArgs& a, const PassCtx& c, const Item& it, int lane) {
+  const bool a0 = lane >= it.c0 && lane <= it.c1 && tile_active(a, c, it.h, it.rt, lane);
+  const bool a1 = lane + 32 >= it.c0 && lane + 32 <= it.c1 && tile_active(a, c, it.h, it.rt, lane + 32);
   return (uint64_t)__ballot_sync(0xffffffffu, a0) | ((uint64_t)__ballot_sync(0xffffffffu, a1) << 32);
 }
 
@@ -350,6 +378,8 @@ pe_sweep_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
   unsigned long long* hmass = reinterpret_cast<unsigned long long*>(sgen + OFF_HMASS);
   float2* xch = reinterpret_cast<float2*>(sgen + OFF_XCH);
   float2* rows_sm = reinterpret_cast<float2*>(sgen + OFF_ROW);
+  int* live_sm = reinterpret_cast<int*>(sgen + OFF_LIVE);
+  const int* live = live_sm + 1;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nbk = MODE == kHist1 ? kHistL1 : MODE == kHist2 ? kHistL2 : 1024;
 
@@ -373,8 +403,19 @@ pe_sweep_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
     hcnt[i] = 0u;
     hmass[i] = 0ull;
   }
+  if (warp == 0) {   // the heads routed PE, in order
+    int cnt = 0;
+    for (int h0 = 0; h0 < a.h_q; h0 += 32) {
+      const bool pe = h0 + lane < a.h_q && a.route[h0 + lane] == 1;
+      const uint32_t bal = __ballot_sync(0xffffffffu, pe);
+      if (pe) live_sm[1 + cnt + __popc(bal & ((1u << lane) - 1u))] = h0 + lane;
+      cnt += __popc(bal);
+    }
+    if (lane == 0) live_sm[0] = cnt;
+  }
   __syncthreads();
   if (*abort_flag) return;   // an earlier kernel failed: do nothing (uniform, before TMEM is taken)
+  const int n_live = live_sm[0];
   if (warp == 1) {
     dev::tmem_alloc(dev::smem_u32(tmem_ptr_smem), kTmemCols);
     dev::tmem_relinquish();
@@ -395,11 +436,11 @@ pe_sweep_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
     int kt = 0;
     bool ok = true;
     PassCtx c;
-    int h, rt;
-    for (int it = 0; ok && item_of(a, blockIdx.x, it, h, rt); ++it) {
-      if (!head_live(a, MODE, h, c)) continue;
-      const uint64_t act = stripe_mask(a, c, h, rt, lane);
-      const int g = h / a.group;
+    Item item;
+    for (int it = 0; ok && item_of(a, live, n_live, MODE, blockIdx.x, it, item); ++it) {
+      if (!head_live(a, MODE, item.h, c)) continue;
+      const uint64_t act = stripe_mask(a, c, item, lane);
+      const int g = item.h / a.group;
       for (int sw = 0; ok && sw < sweeps_of(MODE); ++sw) {
         for (uint64_t m = act; ok && m; m &= m - 1) {
           const int ct = __ffsll((long long)m) - 1;
@@ -434,10 +475,10 @@ pe_sweep_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
     int kt = 0, j = 0, qi = 0;
     bool ok = true;
     PassCtx c;
-    int h, rt;
-    for (int it = 0; ok && item_of(a, blockIdx.x, it, h, rt); ++it) {
-      if (!head_live(a, MODE, h, c)) continue;
-      const uint64_t act = stripe_mask(a, c, h, rt, lane);
+    Item item;
+    for (int it = 0; ok && item_of(a, live, n_live, MODE, blockIdx.x, it, item); ++it) {
+      if (!head_live(a, MODE, item.h, c)) continue;
+      const uint64_t act = stripe_mask(a, c, item, lane);
       if (act == 0) continue;
       if (lane == 0) ok = dev::mbar_wait(bar_addr(sbase, B_QFULL + (qi & 1)), (qi >> 1) & 1, abort_flag, a.status, 42);
       ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -490,7 +531,7 @@ pe_sweep_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
     int j = 0, qi = 0;
     bool ok = true;
     PassCtx c;
-    int h, rt;
+    Item item;
 
     // write the Q-bar rows of stripe (hq, rtq) into TMEM buffer `buf` (this
     // warpgroup's half: hi for warpgroup 0, lo for 1); q = its index among the
@@ -527,11 +568,16 @@ pe_sweep_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
       dev::mbar_arrive(bar_addr(sbase, B_QFULL + buf));
       return true;
     };
-    // next stripe after item `it` with tensor-core work, for the Q prefetch
+    // next item after item `it` with tensor-core work, for the Q prefetch
     auto next_active = [&](int it, int& hn, int& rtn) -> bool {
       PassCtx cn;
-      for (int k = it + 1; item_of(a, blockIdx.x, k, hn, rtn); ++k)
-        if (head_live(a, MODE, hn, cn) && stripe_mask(a, cn, hn, rtn, lane) != 0) return true;
+      Item in;
+      for (int k = it + 1; item_of(a, live, n_live, MODE, blockIdx.x, k, in); ++k)
+        if (head_live(a, MODE, in.h, cn) && stripe_mask(a, cn, in, lane) != 0) {
+          hn = in.h;
+          rtn = in.rt;
+          return true;
+        }
       return false;
     };
     // Quarter q (columns [32q, 32q + 32)) of the S tile j into x; the first
@@ -571,10 +617,11 @@ pe_sweep_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
       if (next_active(-1, h0, rt0)) ok = write_q(h0, rt0, 0);
     }
     int li = -1;   // live stripes so far
-    for (int it = 0; ok && item_of(a, blockIdx.x, it, h, rt); ++it) {
+    for (int it = 0; ok && item_of(a, live, n_live, MODE, blockIdx.x, it, item); ++it) {
+      const int h = item.h, rt = item.rt;
       if (!head_live(a, MODE, h, c)) continue;
       ++li;
-      const uint64_t act_mask = stripe_mask(a, c, h, rt, lane);
+      const uint64_t act_mask = stripe_mask(a, c, item, lane);
       const uint64_t above_mask = (MODE == kMask && !c.all) ? stripe_above(a, c, h, rt, lane) : 0ull;
       const int n_act = __popcll(act_mask);
       if (n_act > 0) {
@@ -750,7 +797,15 @@ pe_sweep_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
           if (!ok) break;
           if (mine && row_ok) a.tie_row[(size_t)h * a.nb + r] = run;
         }
-        for (int ct = 0; MODE != kTies && ct <= rt; ++ct) {
+        // Level 1: a row's entries lie at or below its largest one, inv
+        // (st.y), and in a near-uniform row within a few level-1 buckets of
+        // it; the counts and mass of the four buckets below inv's are kept
+        // per row in registers over the item's tiles (predicated adds) and
+        // reach the shared histogram once, the rest one by one.
+        const uint32_t wbase = __float_as_uint(st.y) >> 8;
+        uint32_t wc0 = 0, wc1 = 0, wc2 = 0, wc3 = 0;
+        unsigned long long wm0 = 0, wm1 = 0, wm2 = 0, wm3 = 0;
+        for (int ct = item.c0; MODE != kTies && ct <= item.c1; ++ct) {
           const bool act = (act_mask >> ct) & 1ull;
           const int last = last_of(ct);
           const int owner = act ? (j & 1) : (ct & 1);
@@ -758,10 +813,47 @@ pe_sweep_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
             if (act) ++j;
             continue;
           }
-          if (MODE == kHist1 || MODE == kHist2) {
-            const int shift_p = MODE == kHist1 ? 20 : 8;
-            const int shift_b = MODE == kHist1 ? 8 : 0;
-            const uint32_t bmask = MODE == kHist1 ? 0xFFFu : 0xFFu;
+          if (MODE == kHist1) {
+#pragma unroll 1
+            for (int qq = 0; qq < 4; ++qq) {
+              if (!load_q(qq, x)) {
+                ok = false;
+                break;
+              }
+              const int lastc = last - 32 * qq;
+              bool far = false;
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                const bool valid = i <= lastc;
+                const float v = dev::ex2(valid ? x[i] - st.x : -INFINITY) * st.y;
+                const uint32_t key = __float_as_uint(v);
+                const bool in = valid && (key >> 20) == c.prefix;
+                const uint32_t off = in ? wbase - (key >> 8) : 0xFFFFFFFFu;
+                const unsigned long long fx = mass_fixed(v);
+                wc0 += off == 0 ? 1u : 0u;
+                wm0 += off == 0 ? fx : 0ull;
+                wc1 += off == 1 ? 1u : 0u;
+                wm1 += off == 1 ? fx : 0ull;
+                wc2 += off == 2 ? 1u : 0u;
+                wm2 += off == 2 ? fx : 0ull;
+                wc3 += off == 3 ? 1u : 0u;
+                wm3 += off == 3 ? fx : 0ull;
+                far = far || (in && off > 3u);
+              }
+              if (__any_sync(0xffffffffu, far)) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                  const bool valid = i <= lastc;
+                  const float v = dev::ex2(valid ? x[i] - st.x : -INFINITY) * st.y;
+                  const uint32_t key = __float_as_uint(v);
+                  if (valid && (key >> 20) == c.prefix && wbase - (key >> 8) > 3u)
+                    hist_add(hcnt, hmass, (key >> 8) & 0xFFFu, 1u, mass_fixed(v));
+                }
+              }
+            }
+            if (!ok) break;
+            ++j;
+          } else if (MODE == kHist2) {
 #pragma unroll 1
             for (int qq = 0; qq < 4; ++qq) {
               if (!load_q(qq, x)) {
@@ -774,8 +866,7 @@ pe_sweep_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
                 const bool valid = i <= lastc;
                 const float v = dev::ex2(valid ? x[i] - st.x : -INFINITY) * st.y;
                 const uint32_t key = __float_as_uint(v);
-                if (valid && (key >> shift_p) == c.prefix)
-                  hist_add(hcnt, hmass, (key >> shift_b) & bmask, 1u, mass_fixed(v));
+                if (valid && (key >> 8) == c.prefix) hist_add(hcnt, hmass, key & 0xFFu, 1u, mass_fixed(v));
               }
             }
             if (!ok) break;
@@ -831,7 +922,14 @@ pe_sweep_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
           }
         }
         if (!ok) break;
-        if (MODE == kHist1 || MODE == kHist2) {
+        if (MODE == kHist1 && n_act > 0) {
+          const uint32_t cs[4] = {wc0, wc1, wc2, wc3};
+          const unsigned long long ms[4] = {wm0, wm1, wm2, wm3};
+#pragma unroll
+          for (int w = 0; w < 4; ++w)
+            if (cs[w]) hist_add(hcnt, hmass, (wbase - w) & 0xFFFu, cs[w], ms[w]);
+        }
+        if ((MODE == kHist1 || MODE == kHist2) && n_act > 0) {
           if (!flush_hist(h)) {
             ok = false;
             break;
@@ -839,12 +937,12 @@ pe_sweep_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
         }
         if (MODE == kMask) {
           // words of the columns beyond this stripe's diagonal tile are zero
-          if (wg == 0 && row_ok)
+          if (item.last && wg == 0 && row_ok)
             for (int word = (rt + 1) * 4; word < a.words; ++word) mrow[word] = 0u;
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) kept += __shfl_xor_sync(0xffffffffu, kept, o);
           if (lane == 0 && kept) atomicAdd(reinterpret_cast<unsigned long long*>(a.pe_count + h), kept);
-          if (rt == 0 && wg == 0 && lr == 0) a.pe_cut[h] = c.all ? 0.f : __uint_as_float(c.cut);
+          if (rt == 0 && item.c0 == 0 && wg == 0 && lr == 0) a.pe_cut[h] = c.all ? 0.f : __uint_as_float(c.cut);
         }
       }
       if (n_act > 0) ++qi;

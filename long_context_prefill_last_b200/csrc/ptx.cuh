@@ -160,6 +160,63 @@ __device__ __forceinline__ void umma_commit(uint32_t bar) {
                : "memory");
 }
 
+// Warp-wide forms: the whole warp executes them (so the descriptors stay
+// warp-uniform) and one elected lane issues the instruction.
+//
+// Eight K = 16 steps of D (+)= A * B with A and B K-major, 128-byte swizzled
+// in shared memory (a 128 x 128 bf16 operand as two 64-column halves): step kk
+// starts (kk / 4) halves and (kk % 4) * 32 bytes in, i.e. the descriptors'
+// start-address fields (16-byte units) advance by (kk / 4) * 1024 + (kk % 4) * 2.
+// The first step accumulates when `accumulate` is nonzero, the rest always.
+#define CRISP_SS_STEP(OFF) \
+  "add.s64 a, %1, " #OFF ";\n\tadd.s64 b, %2, " #OFF ";\n\t@e tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, pt;\n\t"
+__device__ __forceinline__ void umma_ss8_w(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                           uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred e, p0, pt;\n\t.reg .b32 r;\n\t.reg .b64 a, b;\n\t"
+      "elect.sync r|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p0, %4, 0;\n\t"
+      "setp.eq.b32 pt, %4, %4;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p0;\n\t"
+      CRISP_SS_STEP(2) CRISP_SS_STEP(4) CRISP_SS_STEP(6) CRISP_SS_STEP(1024)
+      CRISP_SS_STEP(1026) CRISP_SS_STEP(1028) CRISP_SS_STEP(1030)
+      "}"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+#undef CRISP_SS_STEP
+
+// Eight K = 16 steps of D (+)= A * B with A in tensor memory (bf16 pairs, 8
+// columns per step) and B MN-major, 128-byte swizzled in shared memory (16
+// K-rows of 128 bytes per step: the start-address field advances by 128).
+#define CRISP_TS_STEP(COL, OFF) \
+  "add.u32 t, %1, " #COL ";\n\tadd.s64 b, %2, " #OFF ";\n\t@e tcgen05.mma.cta_group::1.kind::f16 [%0], [t], b, %3, pt;\n\t"
+__device__ __forceinline__ void umma_ts8_w(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                           uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred e, p0, pt;\n\t.reg .b32 r, t;\n\t.reg .b64 b;\n\t"
+      "elect.sync r|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p0, %4, 0;\n\t"
+      "setp.eq.b32 pt, %4, %4;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p0;\n\t"
+      CRISP_TS_STEP(8, 128) CRISP_TS_STEP(16, 256) CRISP_TS_STEP(24, 384) CRISP_TS_STEP(32, 512)
+      CRISP_TS_STEP(40, 640) CRISP_TS_STEP(48, 768) CRISP_TS_STEP(56, 896)
+      "}"
+      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+#undef CRISP_TS_STEP
+
+// Commit (warp-wide form): one elected lane arrives on the mbarrier once every
+// tcgen05.mma issued so far by this thread completes.
+__device__ __forceinline__ void umma_commit_w(uint32_t bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t.reg .b32 r;\n\t"
+      "elect.sync r|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(bar)
+      : "memory");
+}
+
 // Instruction descriptor: bf16 x bf16 -> fp32, M x N, A K-major, B K-major or MN-major.
 __host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N, bool b_mn_major) {
   return (1u << 4)                          // D format: f32
