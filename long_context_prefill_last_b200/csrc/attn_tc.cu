@@ -13,7 +13,8 @@
 // or two KV heads' keys and values, which stay in L2 between them (at
 // 512K tokens this cut DRAM reads from 5.0 TB to 1.9 TB per launch). 12 warps in three warpgroups:
 //   warp 0       TMA producer: Q_A, Q_B once, then K (3-stage ring) and V (2-stage ring)
-//   warp 1       TMEM allocation; one thread issues every tcgen05.mma
+//   warp 1       TMEM allocation; walks the schedule warp-wide (descriptors stay
+//                warp-uniform) and one elected lane issues every tcgen05.mma
 //   warps 2, 3   idle (they complete the first warpgroup)
 //   warps 4..7   softmax of tile A, warps 8..11 softmax of tile B (row = TMEM lane)
 // The first warpgroup gives registers to the softmax warpgroups
@@ -123,10 +124,6 @@ __device__ __forceinline__ void mask_row(float (&s)[128], int kind, int r) {
 #pragma unroll
     for (int c = 0; c < 128; ++c) s[c] = c > r ? s[c] : -INFINITY;
   }
-}
-
-__device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile_base, int kk) {
-  return dev::smem_desc_sw128(tile_base + (kk >> 2) * kHalfBytes + (kk & 3) * 32, 16, 1024);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -254,83 +251,82 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc_qk = dev::umma_idesc_bf16(128, 128, false);
-      const uint32_t idesc_pv = dev::umma_idesc_bf16(128, 128, true);
-      const uint32_t S[2] = {tmem + 0u, tmem + 128u};
-      const uint32_t O[2] = {tmem + 256u, tmem + 384u};
-      const uint32_t QS[2] = {sbase + OFF_QA, sbase + OFF_QB};
-      int kx[2] = {0, 0};   // P.V issued per tile
-      auto qk = [&](int x, int u) {
-        const uint32_t kb = sbase + OFF_K + (u % kKStages) * kTileBytes;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          dev::umma_ss(S[x], kmajor_desc(QS[x], kk), kmajor_desc(kb, kk), idesc_qk, kk > 0 ? 1u : 0u);
-        dev::umma_commit(bar_addr(sbase, B_SFULL + x));
-      };
-      auto pv = [&](int x, int u) -> bool {
-        if (!dev::mbar_wait(bar_addr(sbase, B_PFULL + x), kx[x] & 1, abort_flag, a.status, 4 + x)) return false;
-        dev::tc_fence_after();
-        const uint32_t vb = sbase + OFF_V + (u % kVStages) * kTileBytes;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          dev::umma_ts(O[x], S[x] + kk * 8, dev::smem_desc_sw128(vb + kk * 2048, kHalfBytes, 1024), idesc_pv,
-                       (kx[x] > 0 || kk > 0) ? 1u : 0u);
-        ++kx[x];
-        return true;
-      };
-      bool ok = dev::mbar_wait(bar_addr(sbase, B_Q), 0, abort_flag, a.status, 3);
-      int t = 0, ka = 0, kb = 0;
-      bool have = ok && sc.next(t, ka, kb);
-      if (have) {
-        ok = dev::mbar_wait(bar_addr(sbase, B_KFULL + 0), 0, abort_flag, a.status, 6);
-        dev::tc_fence_after();
-        if (ok && ka != dev::kSkip) qk(0, 0);
-      }
-      int u = 0;
-      while (ok && have) {
-        // lookahead: the tile after u
-        int t2 = t + 1, ka2 = 0, kb2 = 0;
-        const bool have2 = sc.next(t2, ka2, kb2);
-        if (kb != dev::kSkip) qk(1, u);
-        dev::umma_commit(bar_addr(sbase, B_KEMPTY + u % kKStages));
-        if (!dev::mbar_wait(bar_addr(sbase, B_VFULL + u % kVStages), (u / kVStages) & 1, abort_flag, a.status, 7)) {
-          ok = false;
-          break;
-        }
-        dev::tc_fence_after();
-        if (ka != dev::kSkip && !pv(0, u)) {
-          ok = false;
-          break;
-        }
-        if (have2) {
-          if (!dev::mbar_wait(bar_addr(sbase, B_KFULL + (u + 1) % kKStages), ((u + 1) / kKStages) & 1, abort_flag,
-                              a.status, 8)) {
-            ok = false;
-            break;
-          }
-          dev::tc_fence_after();
-          if (ka2 != dev::kSkip) qk(0, u + 1);
-        }
-        if (kb != dev::kSkip && !pv(1, u)) {
-          ok = false;
-          break;
-        }
-        dev::umma_commit(bar_addr(sbase, B_VEMPTY + u % kVStages));
-        t = t2;
-        ka = ka2;
-        kb = kb2;
-        have = have2;
-        ++u;
-      }
-      if (ok) {
-        dev::umma_commit(bar_addr(sbase, B_DONE + 0));
-        dev::umma_commit(bar_addr(sbase, B_DONE + 1));
-      }
-      // every MMA issued must complete before TMEM is released
-      dev::umma_commit(bar_addr(sbase, B_DRAIN));
-      dev::mbar_drain(bar_addr(sbase, B_DRAIN), 0);
+    // The whole warp walks the schedule and waits (the descriptors stay
+    // warp-uniform); one elected lane issues every tcgen05.mma and commit.
+    const uint32_t idesc_qk = dev::umma_idesc_bf16(128, 128, false);
+    const uint32_t idesc_pv = dev::umma_idesc_bf16(128, 128, true);
+    // descriptors of the first K stage and V stage; stages and Q_B are
+    // whole tiles further (kTileBytes / 16 in the start-address field)
+    const uint64_t QD0 = dev::smem_desc_sw128(sbase + OFF_QA, 16, 1024);
+    const uint64_t KD0 = dev::smem_desc_sw128(sbase + OFF_K, 16, 1024);
+    const uint64_t VD0 = dev::smem_desc_sw128(sbase + OFF_V, kHalfBytes, 1024);
+    int kx0 = 0, kx1 = 0;   // P.V issued per tile
+    auto qk = [&](int x, int u) {
+      dev::umma_ss8_w(tmem + (uint32_t)x * 128u, QD0 + (uint64_t)(x * (kTileBytes >> 4)),
+                      KD0 + (uint64_t)((u % kKStages) * (kTileBytes >> 4)), idesc_qk, 0u);
+      dev::umma_commit_w(bar_addr(sbase, B_SFULL + x));
+    };
+    auto pv = [&](int x, int u) -> bool {
+      const int kx = x == 0 ? kx0 : kx1;
+      if (!warp_wait(bar_addr(sbase, B_PFULL + x), kx & 1, abort_flag, a.status, 4 + x)) return false;
+      dev::tc_fence_after();
+      dev::umma_ts8_w(tmem + 256u + (uint32_t)x * 128u, tmem + (uint32_t)x * 128u,
+                      VD0 + (uint64_t)((u % kVStages) * (kTileBytes >> 4)), idesc_pv, kx > 0 ? 1u : 0u);
+      if (x == 0) ++kx0; else ++kx1;
+      return true;
+    };
+    bool ok = warp_wait(bar_addr(sbase, B_Q), 0, abort_flag, a.status, 3);
+    int t = 0, ka = 0, kb = 0;
+    bool have = ok && sc.next(t, ka, kb);
+    if (have) {
+      ok = warp_wait(bar_addr(sbase, B_KFULL + 0), 0, abort_flag, a.status, 6);
+      dev::tc_fence_after();
+      if (ok && ka != dev::kSkip) qk(0, 0);
     }
+    int u = 0;
+    while (ok && have) {
+      // lookahead: the tile after u
+      int t2 = t + 1, ka2 = 0, kb2 = 0;
+      const bool have2 = sc.next(t2, ka2, kb2);
+      if (kb != dev::kSkip) qk(1, u);
+      dev::umma_commit_w(bar_addr(sbase, B_KEMPTY + u % kKStages));
+      if (!warp_wait(bar_addr(sbase, B_VFULL + u % kVStages), (u / kVStages) & 1, abort_flag, a.status, 7)) {
+        ok = false;
+        break;
+      }
+      dev::tc_fence_after();
+      if (ka != dev::kSkip && !pv(0, u)) {
+        ok = false;
+        break;
+      }
+      if (have2) {
+        if (!warp_wait(bar_addr(sbase, B_KFULL + (u + 1) % kKStages), ((u + 1) / kKStages) & 1, abort_flag,
+                       a.status, 8)) {
+          ok = false;
+          break;
+        }
+        dev::tc_fence_after();
+        if (ka2 != dev::kSkip) qk(0, u + 1);
+      }
+      if (kb != dev::kSkip && !pv(1, u)) {
+        ok = false;
+        break;
+      }
+      dev::umma_commit_w(bar_addr(sbase, B_VEMPTY + u % kVStages));
+      t = t2;
+      ka = ka2;
+      kb = kb2;
+      have = have2;
+      ++u;
+    }
+    if (ok) {
+      dev::umma_commit_w(bar_addr(sbase, B_DONE + 0));
+      dev::umma_commit_w(bar_addr(sbase, B_DONE + 1));
+    }
+    // every MMA issued must complete before TMEM is released
+    dev::umma_commit_w(bar_addr(sbase, B_DRAIN));
+    dev::mbar_drain(bar_addr(sbase, B_DRAIN), 0);
+    __syncwarp();
   } else if (warp >= 4) {
     // ---------------------------------------------------------------- softmax warps
     dev::regs_acquire<kRegsSoftmax>();
