@@ -206,10 +206,6 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
   return __all_sync(0xffffffffu, ok);
 }
 
-__device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile_base, int kk) {
-  return dev::smem_desc_sw128(tile_base + (kk >> 2) * kHalfBytes + (kk & 3) * 32, 16, 1024);
-}
-
 // The value of one map entry from its log2-domain logit and its row's (m, inv);
 // every pass evaluates exactly this expression, so they all see the same bits.
 __device__ __forceinline__ float entry_value(float l, float m, float inv) { return dev::ex2(l - m) * inv; }
@@ -470,8 +466,10 @@ pe_sweep_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
-    // the whole warp walks the stripes; lane 0 issues every tcgen05.mma
+    // the whole warp walks the items and waits (descriptors stay
+    // warp-uniform); one elected lane issues every tcgen05.mma and commit
     const uint32_t idesc = dev::umma_idesc_bf16(128, 128, false);
+    const uint64_t KD0 = dev::smem_desc_sw128(sbase + OFF_K, 16, 1024);
     int kt = 0, j = 0, qi = 0;
     bool ok = true;
     PassCtx c;
@@ -480,45 +478,39 @@ pe_sweep_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
       if (!head_live(a, MODE, item.h, c)) continue;
       const uint64_t act = stripe_mask(a, c, item, lane);
       if (act == 0) continue;
-      if (lane == 0) ok = dev::mbar_wait(bar_addr(sbase, B_QFULL + (qi & 1)), (qi >> 1) & 1, abort_flag, a.status, 42);
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) break;
+      if (!warp_wait(bar_addr(sbase, B_QFULL + (qi & 1)), (qi >> 1) & 1, abort_flag, a.status, 42)) {
+        ok = false;
+        break;
+      }
       dev::tc_fence_after();
       const uint32_t qcol = tmem + 256u + (uint32_t)(qi & 1) * 128u;
       for (int sw = 0; ok && sw < sweeps_of(MODE); ++sw) {
         for (uint64_t m = act; ok && m; m &= m - 1) {
           const int s = kt % kStages, buf = j & 1;
-          if (lane == 0) {
-            ok = dev::mbar_wait(bar_addr(sbase, B_KFULL + s), (kt / kStages) & 1, abort_flag, a.status, 43);
-            if (ok && j >= 2)
-              ok = dev::mbar_wait(bar_addr(sbase, B_SEMPTY + buf), ((j - 2) >> 1) & 1, abort_flag, a.status, 44);
-            if (ok) {
-              dev::tc_fence_after();
-              const uint32_t kh = sbase + OFF_K + s * 2 * kTileBytes, kl = kh + kTileBytes;
-              const uint32_t d = tmem + (uint32_t)buf * 128u;
-#pragma unroll
-              for (int kk = 0; kk < 8; ++kk)
-                dev::umma_ts(d, qcol + kk * 8, kmajor_desc(kh, kk), idesc, kk > 0 ? 1u : 0u);
-#pragma unroll
-              for (int kk = 0; kk < 8; ++kk) dev::umma_ts(d, qcol + 64 + kk * 8, kmajor_desc(kh, kk), idesc, 1u);
-#pragma unroll
-              for (int kk = 0; kk < 8; ++kk) dev::umma_ts(d, qcol + kk * 8, kmajor_desc(kl, kk), idesc, 1u);
-              dev::umma_commit(bar_addr(sbase, B_SFULL + buf));
-              dev::umma_commit(bar_addr(sbase, B_KEMPTY + s));
-            }
+          ok = warp_wait(bar_addr(sbase, B_KFULL + s), (kt / kStages) & 1, abort_flag, a.status, 43);
+          if (ok && j >= 2)
+            ok = warp_wait(bar_addr(sbase, B_SEMPTY + buf), ((j - 2) >> 1) & 1, abort_flag, a.status, 44);
+          if (ok) {
+            dev::tc_fence_after();
+            // K-bar hi then lo of stage s (each a whole tile further in the start-address field)
+            const uint64_t kh = KD0 + (uint64_t)(s * 2 * (kTileBytes >> 4)), kl = kh + (kTileBytes >> 4);
+            const uint32_t d = tmem + (uint32_t)buf * 128u;
+            dev::umma_ts8k_w(d, qcol, kh, idesc, 0u);        // Qh . Kh
+            dev::umma_ts8k_w(d, qcol + 64, kh, idesc, 1u);   // Ql . Kh
+            dev::umma_ts8k_w(d, qcol, kl, idesc, 1u);        // Qh . Kl
+            dev::umma_commit_w(bar_addr(sbase, B_SFULL + buf));
+            dev::umma_commit_w(bar_addr(sbase, B_KEMPTY + s));
           }
-          ok = __shfl_sync(0xffffffffu, ok, 0);
           ++kt;
           ++j;
         }
       }
-      if (lane == 0) dev::umma_commit(bar_addr(sbase, B_QEMPTY + (qi & 1)));   // this stripe's Q-bar is no longer read
+      dev::umma_commit_w(bar_addr(sbase, B_QEMPTY + (qi & 1)));   // this stripe's Q-bar is no longer read
       ++qi;
     }
-    if (lane == 0) {   // every MMA issued completes before TMEM is released
-      dev::umma_commit(bar_addr(sbase, B_DRAIN));
-      dev::mbar_drain(bar_addr(sbase, B_DRAIN), 0);
-    }
+    // every MMA issued completes before TMEM is released
+    dev::umma_commit_w(bar_addr(sbase, B_DRAIN));
+    dev::mbar_drain(bar_addr(sbase, B_DRAIN), 0);
     __syncwarp();
   } else if (warp >= 4) {
     // ---------------------------------------------------------------- epilogue warpgroups

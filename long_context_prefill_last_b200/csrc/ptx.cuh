@@ -207,6 +207,27 @@ __device__ __forceinline__ void umma_ts8_w(uint32_t d_tmem, uint32_t a_tmem, uin
 }
 #undef CRISP_TS_STEP
 
+// Eight K = 16 steps of D (+)= A * B with A in tensor memory (bf16 pairs, 8
+// columns per step) and B K-major, 128-byte swizzled in shared memory (as in
+// umma_ss8_w: (kk / 4) * 1024 + (kk % 4) * 2 in the start-address field).
+#define CRISP_TSK_STEP(COL, OFF) \
+  "add.u32 t, %1, " #COL ";\n\tadd.s64 b, %2, " #OFF ";\n\t@e tcgen05.mma.cta_group::1.kind::f16 [%0], [t], b, %3, pt;\n\t"
+__device__ __forceinline__ void umma_ts8k_w(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred e, p0, pt;\n\t.reg .b32 r, t;\n\t.reg .b64 b;\n\t"
+      "elect.sync r|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p0, %4, 0;\n\t"
+      "setp.eq.b32 pt, %4, %4;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p0;\n\t"
+      CRISP_TSK_STEP(8, 2) CRISP_TSK_STEP(16, 4) CRISP_TSK_STEP(24, 6) CRISP_TSK_STEP(32, 1024)
+      CRISP_TSK_STEP(40, 1026) CRISP_TSK_STEP(48, 1028) CRISP_TSK_STEP(56, 1030)
+      "}"
+      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+#undef CRISP_TSK_STEP
+
 // Commit (warp-wide form): one elected lane arrives on the mbarrier once every
 // tcgen05.mma issued so far by this thread completes.
 __device__ __forceinline__ void umma_commit_w(uint32_t bar) {
