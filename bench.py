@@ -201,8 +201,15 @@ def kernel_source_hash(names):
 
 # dram__bytes_read.sum + dram__bytes_write.sum per attention launch, measured
 # by ncu on a scaled case of the layer (one KV group, the same n) and scaled by
-# the KV groups; valid only for the kernel source it was taken on.
-MEASURED_TRAFFIC = {}
+# the KV groups; valid only for the kernel source it was taken on. Layer E:
+# a planted group 20193003520 + 530550016 bytes, a Gaussian group
+# 449172130816 + 533790208 bytes; 6 planted and 2 Gaussian groups.
+MEASURED_TRAFFIC = {
+    ("attn_tc_kernel", "E", 1.0, 0.95): {
+        "source_hash": "86614b33db23dd51",
+        "bytes_per_launch": 6 * (20193003520 + 530550016) + 2 * (449172130816 + 533790208),
+    },
+}
 
 
 def load_traffic(kernel, src_hash, config, alpha, gamma):
