@@ -30,7 +30,7 @@ struct WsLayout {
   size_t khi, klo;    // bf16 [h_kv][nt*128][d]      pooled K, hi and lo parts (rows past N_b zero)
   size_t row_stat;    // f32x2 [h_q][N_b]            pooled-map row (maximum, 1 / (sum * N_b)), log2 domain
   size_t tile_kr;     // u32x2 [h_q][nt][nt][4]      (min, max) key of each 32-row quarter of a 128x128 map tile
-  size_t tie_cnt;     // u32 [h_q][N_b][nt]          entries equal to the cut in the row before each tile
+  size_t tie_cnt;     // u32 [h_q][N_b][nt]          entries equal to the cut per (row, tile), then before each tile
   size_t tie_row;     // u32 [h_q][N_b]              entries equal to the cut per row, then offsets
   size_t hist;        // per head: PeHist
   size_t pe_state;    // per head: PeState

@@ -9,9 +9,12 @@
 // gamma. The diagonal block is always kept.
 //
 // How: the cut is found by a three-level radix select over the fp32 bit
-// patterns of the (positive) entries, with per-bucket counts and float64
-// mass, and the map is never stored. Every pass recomputes the pooled
-// logits it needs on the tensor cores: Q-bar * scale and K-bar are split into
+// patterns of the (positive) entries, with per-bucket counts and mass in
+// 64-bit fixed point (exact, so the sums do not depend on their order), and
+// the map is never stored. Every pass evaluates an entry with the same
+// expression, 2^(logit - row max) * row normaliser, so all see the same
+// bits. Every pass recomputes the pooled logits it needs on the tensor
+// cores: Q-bar * scale and K-bar are split into
 // bf16 hi + lo parts and S = Qh.Kh^T + Ql.Kh^T + Qh.Kl^T (the lo.lo term is
 // below fp32 rounding), with Q-bar held in tensor memory as the A operand
 // and K-bar tiles fed by TMA. The passes:
@@ -20,11 +23,11 @@
 //      the entries, their level-0 histogram (bits 31..20) and, per tile, the
 //      smallest and largest key;
 //   2. level 1 (bits 19..8) and level 2 (bits 7..0): only tiles whose key
-//      range meets the prefix found so far are recomputed;
-//   3. ties (only when the cut keeps part of the entries equal to it): one
-//      warpgroup walks each stripe, so every row's count of entries equal to
-//      the cut builds up in a register (its value before each tile is kept),
-//      then the row totals are scanned in flat order;
+//      range meets the prefix found so far are recomputed, in segments of a
+//      few tiles spread over the SMs;
+//   3. ties (only when the cut keeps part of the entries equal to it): each
+//      row's count of entries equal to the cut per tile, then a scan in flat
+//      order (row by row, tile by tile) gives every tile's rank offset;
 //   4. masks: tiles entirely above (below) the cut are written without
 //      recomputation; the rest are recomputed and compared.
 #include <cuda.h>
@@ -50,7 +53,7 @@ struct PeArgs {
   const __nv_bfloat16* qlo;   // [h_q][nb][128]  bf16(Q-bar * scale_log2 - qhi)
   float2* row_stat;           // [h_q][nb]        (row maximum, 1 / (row sum * N_b)), log2 domain
   uint2* tile_kr;             // [h_q][nt][nt][4] (min key, max key) per 32-row quarter of a tile
-  uint32_t* tie_cnt;          // [h_q][nb][nt]    ties of the row in the tiles before each tile
+  uint32_t* tie_cnt;          // [h_q][nb][nt]    ties of the row per tile, then (tie scan) in the tiles before it
   uint32_t* tie_row;          // [h_q][nb]        ties per row, then exclusive offsets in flat order
   PeHist* hist;
   PeState* state;
@@ -175,7 +178,8 @@ constexpr uint32_t kHalfBytes = 128 * 128;
 constexpr int kHistMax = kHistL1;                // largest per-CTA histogram (level 1)
 constexpr uint32_t OFF_K = 0;                                      // [stage][hi, lo] K-bar tiles
 constexpr uint32_t OFF_HCNT = OFF_K + kStages * 2 * kTileBytes;    // u32 [kHistMax]
-constexpr uint32_t OFF_HMASS = OFF_HCNT + kHistMax * 4;            // u64 [kHistMax], fixed-point mass
+constexpr uint32_t OFF_HMASS = OFF_HCNT + kHistMax * 4;            // u64 [kHistMax] fixed-point mass (level 0),
+                                                                   // u32 [kHistMax] low-bit sums (level 1)
 constexpr uint32_t OFF_XCH = OFF_HMASS + kHistMax * 8;             // float2 [128]: row statistics exchange
 constexpr uint32_t OFF_ROW = OFF_XCH + 128 * 8;                    // float2 [128]: (m, inv) of the stripe's rows
 constexpr uint32_t OFF_LIVE = OFF_ROW + 128 * 8;                   // int [kMaxHeads + 1]: count, then PE heads
@@ -206,18 +210,14 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
   return __all_sync(0xffffffffu, ok);
 }
 
-// The value of one map entry from its log2-domain logit and its row's (m, inv);
-// every pass evaluates exactly this expression, so they all see the same bits.
-__device__ __forceinline__ float entry_value(float l, float m, float inv) { return dev::ex2(l - m) * inv; }
-
-// Work items. The statistics and tie passes take whole 128-row stripes (their
-// per-row running values need every tile of a row in order); the level-1,
-// level-2 and mask passes split a stripe into segments of kSegTiles tiles,
-// since the tiles they recompute sit in the few stripes whose rows straddle
-// the prefix or the cut, and whole stripes would leave those to a handful of
-// CTAs.
-constexpr int kSegTiles = 8;
-__device__ __forceinline__ bool segmented(int mode) { return mode == kHist1 || mode == kHist2 || mode == kMask; }
+// Work items. The statistics pass takes whole 128-row stripes (its per-row
+// running maximum and sum need every tile of a row); the later passes split a
+// stripe into segments of 8 tiles, since the tiles they recompute sit in the
+// few stripes whose rows straddle the prefix or the cut, and whole stripes
+// would leave those to a handful of CTAs (2-tile segments measured slower:
+// every item pays for its key ranges and its Q-bar load).
+__device__ __forceinline__ bool segmented(int mode) { return mode != kStatsHist0; }
+__device__ __forceinline__ int seg_tiles(int) { return 8; }
 
 struct Item {
   int h, rt;    // query head, row tile (stripe)
@@ -230,15 +230,16 @@ struct Item {
 __device__ __forceinline__ bool item_of(const PeArgs& a, const int* live, int n_live, int mode, int b, int k,
                                         Item& it) {
   const int G = gridDim.x;   // items per head <= 64 * 8, so every index fits an int
+  const int seg = segmented(mode) ? seg_tiles(mode) : 64;
   int idx = (k & 1) ? (k + 1) * G - 1 - b : k * G + b;
   for (int rt = a.nt - 1; rt >= 0; --rt) {
-    const int cnt = (segmented(mode) ? rt / kSegTiles + 1 : 1) * n_live;
+    const int cnt = (rt / seg + 1) * n_live;
     if (idx < cnt) {
       const int sg = idx / n_live;
       it.h = live[idx - sg * n_live];
       it.rt = rt;
-      it.c0 = segmented(mode) ? sg * kSegTiles : 0;
-      it.c1 = segmented(mode) ? min(rt, it.c0 + kSegTiles - 1) : rt;
+      it.c0 = sg * seg;
+      it.c1 = min(rt, it.c0 + seg - 1);
       it.last = it.c1 == rt;
       return true;
     }
@@ -341,8 +342,21 @@ __device__ __forceinline__ bool epi_sync(uint32_t sbase, uint32_t& phase, volati
   return ok;
 }
 
-// An entry's mass in fixed point (units of 2^-62; entries are at most 1/4).
-__device__ __forceinline__ unsigned long long mass_fixed(float v) { return __float2ull_rn(v * 0x1p62f); }
+// Mass is kept in fixed point, units of 2^-62 (entries are at most 1/4).
+// bucket_mass gives the summed mass of `cnt` entries whose keys agree with
+// `key_base` on every bit above some low bits (zero in key_base) and whose low
+// bits add up to `low`. A positive normal float is (2^23 + mantissa) *
+// 2^(exponent - 150), so the sum is (cnt * (2^23 + high mantissa bits) + low)
+// * 2^(exponent - 150): integer arithmetic, exact for entries of at least
+// 2^-38 (then every entry is a whole number of units); smaller ones are
+// truncated to whole units and subnormal ones count 0. Histograms keep
+// (count, low-bit sum) per bucket in 32-bit integers and convert once.
+__device__ __forceinline__ unsigned long long bucket_mass(uint32_t key_base, uint32_t cnt, unsigned long long low) {
+  const int e = (int)(key_base >> 23);
+  if (e == 0) return 0ull;
+  const unsigned long long x = (unsigned long long)cnt * (0x800000u | (key_base & 0x7FFFFFu)) + low;
+  return e >= 88 ? x << (e - 88) : x >> (88 - e);
+}
 
 __device__ __forceinline__ void hist_add(uint32_t* cnt, unsigned long long* mass, uint32_t b, uint32_t c,
                                          unsigned long long m) {
@@ -372,6 +386,7 @@ pe_sweep_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
   uint32_t* tmem_ptr_smem = reinterpret_cast<uint32_t*>(sgen + OFF_TMEMPTR);
   uint32_t* hcnt = reinterpret_cast<uint32_t*>(sgen + OFF_HCNT);
   unsigned long long* hmass = reinterpret_cast<unsigned long long*>(sgen + OFF_HMASS);
+  uint32_t* hlow = reinterpret_cast<uint32_t*>(sgen + OFF_HMASS);   // level 1: low-bit sums in hmass's space
   float2* xch = reinterpret_cast<float2*>(sgen + OFF_XCH);
   float2* rows_sm = reinterpret_cast<float2*>(sgen + OFF_ROW);
   int* live_sm = reinterpret_cast<int*>(sgen + OFF_LIVE);
@@ -589,16 +604,27 @@ pe_sweep_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
       }
       return true;
     };
+    // add the CTA's histogram of head hh to the head's global one and clear
+    // it; levels 1 and 2 turn (count, low-bit sum) into mass here
     auto flush_hist = [&](int hh) -> bool {
       if (!epi_sync(sbase, epi_phase, abort_flag, a.status)) return false;
       PeHist* gh = a.hist + hh;
       for (int i = threadIdx.x - 128; i < nbk; i += 256) {
         const uint32_t cnt = hcnt[i];
         if (cnt) {
+          unsigned long long m;
+          if (MODE == kHist1) {
+            m = bucket_mass((c.prefix << 20) | ((uint32_t)i << 8), cnt, hlow[i]);
+            hlow[i] = 0u;
+          } else if (MODE == kHist2) {
+            m = bucket_mass((c.prefix << 8) | (uint32_t)i, cnt, 0ull);
+          } else {
+            m = hmass[i];
+            hmass[i] = 0ull;
+          }
           atomicAdd(&gh->count[i], (unsigned long long)cnt);
-          atomicAdd(&gh->mass[i], hmass[i]);
+          atomicAdd(&gh->mass[i], m);
           hcnt[i] = 0u;
-          hmass[i] = 0ull;
         }
       }
       return epi_sync(sbase, epi_phase, abort_flag, a.status);
@@ -608,11 +634,9 @@ pe_sweep_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
       int h0, rt0;
       if (next_active(-1, h0, rt0)) ok = write_q(h0, rt0, 0);
     }
-    int li = -1;   // live stripes so far
     for (int it = 0; ok && item_of(a, live, n_live, MODE, blockIdx.x, it, item); ++it) {
       const int h = item.h, rt = item.rt;
       if (!head_live(a, MODE, h, c)) continue;
-      ++li;
       const uint64_t act_mask = stripe_mask(a, c, item, lane);
       const uint64_t above_mask = (MODE == kMask && !c.all) ? stripe_above(a, c, h, rt, lane) : 0ull;
       const int n_act = __popcll(act_mask);
@@ -691,8 +715,10 @@ pe_sweep_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
           if ((j & 1) != wg) continue;
           const int last = last_of(ct);
           uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+          // per window: entry count and the sum of the low 20 key bits
+          // (at most 128 * 2^20 per thread and tile)
           uint32_t c0 = 0, c1 = 0, c2 = 0, c3 = 0;
-          unsigned long long m0 = 0, m1 = 0, m2 = 0, m3 = 0;
+          uint32_t l0 = 0, l1 = 0, l2 = 0, l3 = 0;
 #pragma unroll 1
           for (int qq = 0; qq < 4; ++qq) {
             if (!load_q(qq, x)) {
@@ -707,36 +733,47 @@ pe_sweep_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
               const float v = dev::ex2(valid ? x[i] - st.x : -INFINITY) * st.y;
               const uint32_t key = __float_as_uint(v);
               kmin = valid ? min(kmin, key) : kmin;
-              kmax = valid ? max(kmax, key) : kmax;
+              kmax = max(kmax, key);   // masked entries are 0.0f (key 0)
               const uint32_t off = valid ? b_base - (key >> 20) : 0xFFFFFFFFu;
-              const unsigned long long fx = mass_fixed(v);
+              const uint32_t low = key & 0xFFFFFu;
               c0 += off == 0 ? 1u : 0u;
-              m0 += off == 0 ? fx : 0ull;
+              l0 += off == 0 ? low : 0u;
               c1 += off == 1 ? 1u : 0u;
-              m1 += off == 1 ? fx : 0ull;
+              l1 += off == 1 ? low : 0u;
               c2 += off == 2 ? 1u : 0u;
-              m2 += off == 2 ? fx : 0ull;
+              l2 += off == 2 ? low : 0u;
               c3 += off == 3 ? 1u : 0u;
-              m3 += off == 3 ? fx : 0ull;
+              l3 += off == 3 ? low : 0u;
               far = far || (valid && off > 3u);
             }
             if (__any_sync(0xffffffffu, far)) {
+              // entries below the window: the lanes of a column that share a
+              // bucket are merged first (count, low-bit sum), so a column whose
+              // rows agree costs one shared atomic instead of 32
 #pragma unroll
               for (int i = 0; i < 32; ++i) {
                 const bool valid = i <= lastc;
-                const float v = dev::ex2(valid ? x[i] - st.x : -INFINITY) * st.y;
-                const uint32_t key = __float_as_uint(v);
-                if (valid && b_base - (key >> 20) > 3u) hist_add(hcnt, hmass, key >> 20, 1u, mass_fixed(v));
+                const uint32_t key = __float_as_uint(dev::ex2(valid ? x[i] - st.x : -INFINITY) * st.y);
+                const bool out = valid && b_base - (key >> 20) > 3u;
+                const uint32_t outs = __ballot_sync(0xffffffffu, out);
+                if (out) {
+                  const uint32_t b = key >> 20;
+                  const uint32_t grp = __match_any_sync(outs, b);
+                  const uint32_t lsum = __reduce_add_sync(grp, key & 0xFFFFFu);
+                  const uint32_t cnt = __popc(grp);
+                  if (lane == __ffs(grp) - 1) hist_add(hcnt, hmass, b, cnt, bucket_mass(b << 20, cnt, lsum));
+                }
               }
             }
           }
           if (!ok) break;
           const uint32_t cs[4] = {warp_sum_u32(c0), warp_sum_u32(c1), warp_sum_u32(c2), warp_sum_u32(c3)};
-          const unsigned long long ms[4] = {warp_sum_u64(m0), warp_sum_u64(m1), warp_sum_u64(m2), warp_sum_u64(m3)};
+          const unsigned long long ls[4] = {warp_sum_u64(l0), warp_sum_u64(l1), warp_sum_u64(l2), warp_sum_u64(l3)};
           if (lane == 0) {
 #pragma unroll
             for (int w = 0; w < 4; ++w)
-              if (cs[w] && b_base >= (uint32_t)w) hist_add(hcnt, hmass, b_base - w, cs[w], ms[w]);
+              if (cs[w] && b_base >= (uint32_t)w)
+                hist_add(hcnt, hmass, b_base - w, cs[w], bucket_mass((b_base - w) << 20, cs[w], ls[w]));
           }
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) {
@@ -756,19 +793,51 @@ pe_sweep_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
         uint32_t* trow = a.tie_cnt + ((size_t)h * a.nb + (row_ok ? r : 0)) * a.nt;
         unsigned long long kept = 0;
         if (MODE == kTies) {
-          // warpgroup li % 2 takes every tile of this stripe, so each row's
-          // count of entries equal to the cut builds up in one register
-          const bool mine = (li & 1) == wg;
-          uint32_t run = 0;
-          for (int ct = 0; ct <= rt; ++ct) {
+          // each row's count of entries equal to the cut, per tile; the tie
+          // scan turns them into running counts in flat order
+          for (int ct = item.c0; ct <= item.c1; ++ct) {
             const bool act = (act_mask >> ct) & 1ull;
-            if (!mine) {
+            const int owner = act ? (j & 1) : (ct & 1);
+            if (owner != wg) {
               if (act) ++j;
               continue;
             }
-            if (row_ok) trow[ct] = run;
-            if (!act) continue;
-            const int last = last_of(ct);
+            uint32_t cnt = 0;
+            if (act) {
+              const int last = last_of(ct);
+#pragma unroll 1
+              for (int qq = 0; qq < 4; ++qq) {
+                if (!load_q(qq, x)) {
+                  ok = false;
+                  break;
+                }
+                const int lastc = last - 32 * qq;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                  const bool valid = i <= lastc;
+                  const uint32_t key = __float_as_uint(dev::ex2(valid ? x[i] - st.x : -INFINITY) * st.y);
+                  cnt += (valid && key == c.cut) ? 1u : 0u;
+                }
+              }
+              if (!ok) break;
+              ++j;
+            }
+            if (row_ok) trow[ct] = cnt;
+          }
+          if (!ok) break;
+        }
+        // Levels 1 and 2 keep, per bucket of the shared histogram, the entry
+        // count and (level 1) the sum of the key bits below the bucket (8
+        // bits), both 32-bit shared atomics; flush_hist turns them into mass.
+        for (int ct = item.c0; MODE != kTies && ct <= item.c1; ++ct) {
+          const bool act = (act_mask >> ct) & 1ull;
+          const int last = last_of(ct);
+          const int owner = act ? (j & 1) : (ct & 1);
+          if (owner != wg || (!act && (MODE == kHist1 || MODE == kHist2))) {
+            if (act) ++j;
+            continue;
+          }
+          if (MODE == kHist1 || MODE == kHist2) {
 #pragma unroll 1
             for (int qq = 0; qq < 4; ++qq) {
               if (!load_q(qq, x)) {
@@ -780,85 +849,14 @@ pe_sweep_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
               for (int i = 0; i < 32; ++i) {
                 const bool valid = i <= lastc;
                 const uint32_t key = __float_as_uint(dev::ex2(valid ? x[i] - st.x : -INFINITY) * st.y);
-                run += (valid && key == c.cut) ? 1u : 0u;
-              }
-            }
-            if (!ok) break;
-            ++j;
-          }
-          if (!ok) break;
-          if (mine && row_ok) a.tie_row[(size_t)h * a.nb + r] = run;
-        }
-        // Level 1: a row's entries lie at or below its largest one, inv
-        // (st.y), and in a near-uniform row within a few level-1 buckets of
-        // it; the counts and mass of the four buckets below inv's are kept
-        // per row in registers over the item's tiles (predicated adds) and
-        // reach the shared histogram once, the rest one by one.
-        const uint32_t wbase = __float_as_uint(st.y) >> 8;
-        uint32_t wc0 = 0, wc1 = 0, wc2 = 0, wc3 = 0;
-        unsigned long long wm0 = 0, wm1 = 0, wm2 = 0, wm3 = 0;
-        for (int ct = item.c0; MODE != kTies && ct <= item.c1; ++ct) {
-          const bool act = (act_mask >> ct) & 1ull;
-          const int last = last_of(ct);
-          const int owner = act ? (j & 1) : (ct & 1);
-          if (owner != wg || (!act && (MODE == kHist1 || MODE == kHist2))) {
-            if (act) ++j;
-            continue;
-          }
-          if (MODE == kHist1) {
-#pragma unroll 1
-            for (int qq = 0; qq < 4; ++qq) {
-              if (!load_q(qq, x)) {
-                ok = false;
-                break;
-              }
-              const int lastc = last - 32 * qq;
-              bool far = false;
-#pragma unroll
-              for (int i = 0; i < 32; ++i) {
-                const bool valid = i <= lastc;
-                const float v = dev::ex2(valid ? x[i] - st.x : -INFINITY) * st.y;
-                const uint32_t key = __float_as_uint(v);
-                const bool in = valid && (key >> 20) == c.prefix;
-                const uint32_t off = in ? wbase - (key >> 8) : 0xFFFFFFFFu;
-                const unsigned long long fx = mass_fixed(v);
-                wc0 += off == 0 ? 1u : 0u;
-                wm0 += off == 0 ? fx : 0ull;
-                wc1 += off == 1 ? 1u : 0u;
-                wm1 += off == 1 ? fx : 0ull;
-                wc2 += off == 2 ? 1u : 0u;
-                wm2 += off == 2 ? fx : 0ull;
-                wc3 += off == 3 ? 1u : 0u;
-                wm3 += off == 3 ? fx : 0ull;
-                far = far || (in && off > 3u);
-              }
-              if (__any_sync(0xffffffffu, far)) {
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                  const bool valid = i <= lastc;
-                  const float v = dev::ex2(valid ? x[i] - st.x : -INFINITY) * st.y;
-                  const uint32_t key = __float_as_uint(v);
-                  if (valid && (key >> 20) == c.prefix && wbase - (key >> 8) > 3u)
-                    hist_add(hcnt, hmass, (key >> 8) & 0xFFFu, 1u, mass_fixed(v));
+                if (MODE == kHist1) {
+                  if (valid && (key >> 20) == c.prefix) {
+                    atomicAdd(&hcnt[(key >> 8) & 0xFFFu], 1u);
+                    atomicAdd(&hlow[(key >> 8) & 0xFFFu], key & 0xFFu);
+                  }
+                } else if (valid && (key >> 8) == c.prefix) {
+                  atomicAdd(&hcnt[key & 0xFFu], 1u);
                 }
-              }
-            }
-            if (!ok) break;
-            ++j;
-          } else if (MODE == kHist2) {
-#pragma unroll 1
-            for (int qq = 0; qq < 4; ++qq) {
-              if (!load_q(qq, x)) {
-                ok = false;
-                break;
-              }
-              const int lastc = last - 32 * qq;
-#pragma unroll
-              for (int i = 0; i < 32; ++i) {
-                const bool valid = i <= lastc;
-                const float v = dev::ex2(valid ? x[i] - st.x : -INFINITY) * st.y;
-                const uint32_t key = __float_as_uint(v);
-                if (valid && (key >> 8) == c.prefix) hist_add(hcnt, hmass, key & 0xFFu, 1u, mass_fixed(v));
               }
             }
             if (!ok) break;
@@ -914,13 +912,6 @@ pe_sweep_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
           }
         }
         if (!ok) break;
-        if (MODE == kHist1 && n_act > 0) {
-          const uint32_t cs[4] = {wc0, wc1, wc2, wc3};
-          const unsigned long long ms[4] = {wm0, wm1, wm2, wm3};
-#pragma unroll
-          for (int w = 0; w < 4; ++w)
-            if (cs[w]) hist_add(hcnt, hmass, (wbase - w) & 0xFFFu, cs[w], ms[w]);
-        }
         if ((MODE == kHist1 || MODE == kHist2) && n_act > 0) {
           if (!flush_hist(h)) {
             ok = false;
@@ -1076,6 +1067,29 @@ __global__ void __launch_bounds__(1024) pe_tie_scan_kernel(PeArgs a) {
   uint32_t* rows = a.tie_row + (size_t)h * a.nb;
   const int per = (a.nb + 1023) / 1024;
   const int lo = threadIdx.x * per, hi = min(a.nb, lo + per);
+  // per row (one warp, lanes over tiles): the tie counts of its tiles
+  // c <= r / 128 become running counts (ties before each tile), the row's
+  // total goes to rows[r]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int r = warp; r < a.nb; r += 32) {
+    uint32_t* t = a.tie_cnt + ((size_t)h * a.nb + r) * a.nt;
+    const int ntile = r / 128 + 1;
+    uint32_t carry = 0;
+    for (int c0 = 0; c0 < ntile; c0 += 32) {
+      const int ct = c0 + lane;
+      const uint32_t v = ct < ntile ? t[ct] : 0u;
+      uint32_t incl = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      if (ct < ntile) t[ct] = carry + incl - v;
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) rows[r] = carry;
+  }
+  __syncthreads();
   unsigned long long s = 0;
   for (int r = lo; r < hi; ++r) s += rows[r];
   part[threadIdx.x] = s;
