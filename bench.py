@@ -54,8 +54,8 @@ METRIC = "sparse-prefill attention ms/layer & speedup vs in-run dense kernel, 12
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 PAGES_SPEEDUP_512K = 5.30   # the pages' figure on a single H100 (context only)
 # kernels of one crisp_select: proxy 1, finalise 2, VS select 1,
-# PE 10 (pool, 5 sweeps, 3 bucket searches, tie scan)
-SELECT_KERNELS = 14
+# PE 12 (pool, 5 sweeps, 3 bucket searches, tie rows, tie scan, mask fill)
+SELECT_KERNELS = 16
 SWEEP = [(1.0, 0.95), (1.0, 0.97), (1.25, 0.95), (1.25, 0.97), (1.5, 0.95), (1.5, 0.97)]
 ALL_CONFIGS = ["A", "B", "C", "D", "E"]
 # FP32 lanes per SM (the CUDA-core attention of fp32 layers is bound by FFMA issue)

@@ -28,8 +28,8 @@
 //   3. ties (only when the cut keeps part of the entries equal to it): each
 //      row's count of entries equal to the cut per tile, then a scan in flat
 //      order (row by row, tile by tile) gives every tile's rank offset;
-//   4. masks: tiles entirely above (below) the cut are written without
-//      recomputation; the rest are recomputed and compared.
+//   4. masks: a fill kernel writes the tiles entirely above (below) the cut
+//      without recomputation; the sweep recomputes the tiles the cut crosses.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
@@ -312,22 +312,6 @@ __device__ __forceinline__ bool tile_active(const PeArgs& a, const PassCtx& c, i
 __device__ __forceinline__ uint64_t stripe_mask(const PeArgs& a, const PassCtx& c, const Item& it, int lane) {
   const bool a0 = lane >= it.c0 && lane <= it.c1 && tile_active(a, c, it.h, it.rt, lane);
   const bool a1 = lane + 32 >= it.c0 && lane + 32 <= it.c1 && tile_active(a, c, it.h, it.rt, lane + 32);
-  return (uint64_t)__ballot_sync(0xffffffffu, a0) | ((uint64_t)__ballot_sync(0xffffffffu, a1) << 32);
-}
-
-// The tiles ct <= rt of stripe (h, rt) whose every entry lies above the cut
-// (kept whole by the mask pass without recomputation); warp-wide like stripe_mask.
-__device__ __forceinline__ uint64_t stripe_above(const PeArgs& a, const PassCtx& c, int h, int rt, int lane) {
-  uint32_t kmin, kmax;
-  bool a0 = false, a1 = false;
-  if (lane <= rt) {
-    tile_range(a, h, rt, lane, kmin, kmax);
-    a0 = kmin > c.cut;
-  }
-  if (lane + 32 <= rt) {
-    tile_range(a, h, rt, lane + 32, kmin, kmax);
-    a1 = kmin > c.cut;
-  }
   return (uint64_t)__ballot_sync(0xffffffffu, a0) | ((uint64_t)__ballot_sync(0xffffffffu, a1) << 32);
 }
 
@@ -638,7 +622,6 @@ pe_sweep_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
       const int h = item.h, rt = item.rt;
       if (!head_live(a, MODE, h, c)) continue;
       const uint64_t act_mask = stripe_mask(a, c, item, lane);
-      const uint64_t above_mask = (MODE == kMask && !c.all) ? stripe_above(a, c, h, rt, lane) : 0ull;
       const int n_act = __popcll(act_mask);
       if (n_act > 0) {
         int hn, rtn;
@@ -833,7 +816,7 @@ pe_sweep_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
           const bool act = (act_mask >> ct) & 1ull;
           const int last = last_of(ct);
           const int owner = act ? (j & 1) : (ct & 1);
-          if (owner != wg || (!act && (MODE == kHist1 || MODE == kHist2))) {
+          if (owner != wg || !act) {   // tiles the cut does not cross: pe_mask_fill_kernel
             if (act) ++j;
             continue;
           }
@@ -861,13 +844,9 @@ pe_sweep_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
             }
             if (!ok) break;
             ++j;
-          } else {   // kMask
+          } else {   // kMask, a tile the cut crosses
             uint32_t w[4] = {0u, 0u, 0u, 0u};
-            if (c.all || ((above_mask >> ct) & 1ull)) {   // every entry kept
-#pragma unroll
-              for (int cc = 0; cc < 128; ++cc)
-                if (cc <= last) w[cc >> 5] |= 1u << (cc & 31);
-            } else if (act) {
+            {
               unsigned long long rank =
                   c.partial_ties && row_ok ? (unsigned long long)a.tie_row[(size_t)h * a.nb + r] + trow[ct] : 0ull;
               const int diag = ct == rt ? ncol : -1;
@@ -919,13 +898,9 @@ pe_sweep_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
           }
         }
         if (MODE == kMask) {
-          // words of the columns beyond this stripe's diagonal tile are zero
-          if (item.last && wg == 0 && row_ok)
-            for (int word = (rt + 1) * 4; word < a.words; ++word) mrow[word] = 0u;
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) kept += __shfl_xor_sync(0xffffffffu, kept, o);
           if (lane == 0 && kept) atomicAdd(reinterpret_cast<unsigned long long*>(a.pe_count + h), kept);
-          if (rt == 0 && item.c0 == 0 && wg == 0 && lr == 0) a.pe_cut[h] = c.all ? 0.f : __uint_as_float(c.cut);
         }
       }
       if (n_act > 0) ++qi;
@@ -1058,6 +1033,76 @@ __global__ void __launch_bounds__(1024) pe_find_kernel(PeArgs a, int level) {
 // keeps part of its ties: flat order is row by row, so a tie's rank is its
 // row's offset plus the ties before it in the row (kept per tile by the
 // ties pass). One CTA of 1024 threads per head.
+// Masks of the tiles the cut does not cross, per row of head blockIdx.y (one
+// warp per row, lanes over words): all ones for c <= r in tiles entirely
+// above the cut (every tile when the cut keeps everything), zero in tiles
+// entirely below it and past the diagonal tile, and the diagonal block always
+// kept. Tiles the cut crosses are left to the mask sweep, which decides them
+// with the same tile key ranges. Adds the kept blocks to pe_count.
+__global__ void __launch_bounds__(256) pe_mask_fill_kernel(PeArgs a) {
+  const int h = blockIdx.y;
+  if (a.route[h] != 1) return;
+  const int r = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (r >= a.nb) return;
+  const PeState* st = a.state + h;
+  const bool all = st->all != 0;
+  const uint32_t cut = st->cut_key;
+  const int rt = r >> 7;
+  uint32_t* mrow = a.pe_mask + ((size_t)h * a.nb + r) * a.words;
+  unsigned long long kept = 0;
+  for (int w = lane; w < a.words; w += 32) {
+    const int ct = w >> 2, c0 = w * 32;
+    uint32_t word = 0u;
+    if (ct <= rt) {
+      bool above = all;
+      if (!all) {
+        uint32_t kmin, kmax;
+        tile_range(a, h, rt, ct, kmin, kmax);
+        if (kmin <= cut && kmax >= cut) continue;   // crossed: the mask sweep writes it
+        above = kmin > cut;
+      }
+      const uint32_t upto = r >= c0 + 31 ? 0xFFFFFFFFu : (r < c0 ? 0u : (2u << (r - c0)) - 1u);   // c <= r
+      word = above ? upto : 0u;
+      if (r >= c0 && r < c0 + 32) word |= 1u << (r - c0);   // the diagonal block
+    }
+    mrow[w] = word;
+    kept += __popc(word);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) kept += __shfl_xor_sync(0xffffffffu, kept, o);
+  if (lane == 0 && kept) atomicAdd(reinterpret_cast<unsigned long long*>(a.pe_count + h), kept);
+  if (r == 0 && lane == 0) a.pe_cut[h] = all ? 0.f : __uint_as_float(cut);
+}
+
+// Ties, per row of head blockIdx.y (one warp per row, lanes over tiles): the
+// counts of the tiles c <= r / 128 become running counts (ties in the tiles
+// before each tile) and the row's total goes to tie_row.
+__global__ void __launch_bounds__(1024) pe_tie_rows_kernel(PeArgs a) {
+  const int h = blockIdx.y;
+  if (a.route[h] != 1) return;
+  const PeState* st = a.state + h;
+  if (st->all || st->t_keep >= st->n_ties) return;
+  const int r = blockIdx.x * 32 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (r >= a.nb) return;
+  uint32_t* t = a.tie_cnt + ((size_t)h * a.nb + r) * a.nt;
+  const int ntile = r / 128 + 1;
+  uint32_t carry = 0;
+  for (int c0 = 0; c0 < ntile; c0 += 32) {
+    const int ct = c0 + lane;
+    const uint32_t v = ct < ntile ? t[ct] : 0u;
+    uint32_t incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (ct < ntile) t[ct] = carry + incl - v;
+    carry += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  if (lane == 0) a.tie_row[(size_t)h * a.nb + r] = carry;
+}
+
+// Ties, per head: the row totals become exclusive offsets in flat order.
 __global__ void __launch_bounds__(1024) pe_tie_scan_kernel(PeArgs a) {
   const int h = blockIdx.x;
   if (a.route[h] != 1) return;
@@ -1067,29 +1112,6 @@ __global__ void __launch_bounds__(1024) pe_tie_scan_kernel(PeArgs a) {
   uint32_t* rows = a.tie_row + (size_t)h * a.nb;
   const int per = (a.nb + 1023) / 1024;
   const int lo = threadIdx.x * per, hi = min(a.nb, lo + per);
-  // per row (one warp, lanes over tiles): the tie counts of its tiles
-  // c <= r / 128 become running counts (ties before each tile), the row's
-  // total goes to rows[r]
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int r = warp; r < a.nb; r += 32) {
-    uint32_t* t = a.tie_cnt + ((size_t)h * a.nb + r) * a.nt;
-    const int ntile = r / 128 + 1;
-    uint32_t carry = 0;
-    for (int c0 = 0; c0 < ntile; c0 += 32) {
-      const int ct = c0 + lane;
-      const uint32_t v = ct < ntile ? t[ct] : 0u;
-      uint32_t incl = v;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      if (ct < ntile) t[ct] = carry + incl - v;
-      carry += __shfl_sync(0xffffffffu, incl, 31);
-    }
-    if (lane == 0) rows[r] = carry;
-  }
-  __syncthreads();
   unsigned long long s = 0;
   for (int r = lo; r < hi; ++r) s += rows[r];
   part[threadIdx.x] = s;
@@ -1178,7 +1200,9 @@ cudaError_t launch_pe(const void* q, const void* k, const Shape& s, char* ws, co
   if ((e = launch_sweep<kHist2>(mh, ml, a, grid, st)) != cudaSuccess) return e;
   pe_find_kernel<<<s.h_q, 1024, 0, st>>>(a, 2);
   if ((e = launch_sweep<kTies>(mh, ml, a, grid, st)) != cudaSuccess) return e;
+  pe_tie_rows_kernel<<<dim3((s.nb + 31) / 32, s.h_q), 1024, 0, st>>>(a);
   pe_tie_scan_kernel<<<s.h_q, 1024, 0, st>>>(a);
+  pe_mask_fill_kernel<<<dim3((s.nb + 7) / 8, s.h_q), 256, 0, st>>>(a);
   if ((e = launch_sweep<kMask>(mh, ml, a, grid, st)) != cudaSuccess) return e;
   return cudaGetLastError();
 }
