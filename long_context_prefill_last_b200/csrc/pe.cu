@@ -1033,45 +1033,52 @@ __global__ void __launch_bounds__(1024) pe_find_kernel(PeArgs a, int level) {
 // keeps part of its ties: flat order is row by row, so a tie's rank is its
 // row's offset plus the ties before it in the row (kept per tile by the
 // ties pass). One CTA of 1024 threads per head.
-// Masks of the tiles the cut does not cross, per row of head blockIdx.y (one
-// warp per row, lanes over words): all ones for c <= r in tiles entirely
-// above the cut (every tile when the cut keeps everything), zero in tiles
-// entirely below it and past the diagonal tile, and the diagonal block always
-// kept. Tiles the cut crosses are left to the mask sweep, which decides them
-// with the same tile key ranges. Adds the kept blocks to pe_count.
+// Masks of the tiles the cut does not cross, for stripe blockIdx.x of head
+// blockIdx.y: all ones for c <= r in tiles entirely above the cut (every tile
+// when the cut keeps everything), zero in tiles entirely below it and past
+// the diagonal tile, and the diagonal block always kept. Tiles the cut crosses
+// are left to the mask sweep, which decides them with the same tile key
+// ranges. Each tile is classified once; the stripe's words are then written
+// row by row (coalesced). Adds the kept blocks to pe_count.
 __global__ void __launch_bounds__(256) pe_mask_fill_kernel(PeArgs a) {
-  const int h = blockIdx.y;
+  const int h = blockIdx.y, rt = blockIdx.x;
   if (a.route[h] != 1) return;
-  const int r = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
-  if (r >= a.nb) return;
+  __shared__ int8_t kind[64];   // per tile ct <= rt: 1 above, 0 below, -1 crossed
   const PeState* st = a.state + h;
   const bool all = st->all != 0;
   const uint32_t cut = st->cut_key;
-  const int rt = r >> 7;
-  uint32_t* mrow = a.pe_mask + ((size_t)h * a.nb + r) * a.words;
-  unsigned long long kept = 0;
-  for (int w = lane; w < a.words; w += 32) {
-    const int ct = w >> 2, c0 = w * 32;
-    uint32_t word = 0u;
-    if (ct <= rt) {
-      bool above = all;
-      if (!all) {
-        uint32_t kmin, kmax;
-        tile_range(a, h, rt, ct, kmin, kmax);
-        if (kmin <= cut && kmax >= cut) continue;   // crossed: the mask sweep writes it
-        above = kmin > cut;
-      }
-      const uint32_t upto = r >= c0 + 31 ? 0xFFFFFFFFu : (r < c0 ? 0u : (2u << (r - c0)) - 1u);   // c <= r
-      word = above ? upto : 0u;
-      if (r >= c0 && r < c0 + 32) word |= 1u << (r - c0);   // the diagonal block
+  if (threadIdx.x <= rt) {
+    int8_t k = 1;
+    if (!all) {
+      uint32_t kmin, kmax;
+      tile_range(a, h, rt, threadIdx.x, kmin, kmax);
+      k = (kmin <= cut && kmax >= cut) ? -1 : (kmin > cut ? 1 : 0);
     }
-    mrow[w] = word;
-    kept += __popc(word);
+    kind[threadIdx.x] = k;
+  }
+  __syncthreads();
+  const int r_end = min(rt * 128 + 128, a.nb);
+  unsigned long long kept = 0;
+  // one warp per row, lanes over the row's words
+  for (int r = rt * 128 + (threadIdx.x >> 5); r < r_end; r += 8) {
+    uint32_t* mrow = a.pe_mask + ((size_t)h * a.nb + r) * a.words;
+    for (int w = threadIdx.x & 31; w < a.words; w += 32) {
+      const int ct = w >> 2, c0 = w * 32;
+      uint32_t word = 0u;
+      if (ct <= rt) {
+        if (kind[ct] < 0) continue;   // crossed: the mask sweep writes it
+        const uint32_t upto = r >= c0 + 31 ? 0xFFFFFFFFu : (r < c0 ? 0u : (2u << (r - c0)) - 1u);   // c <= r
+        word = kind[ct] > 0 ? upto : 0u;
+        if (r >= c0 && r < c0 + 32) word |= 1u << (r - c0);   // the diagonal block
+      }
+      mrow[w] = word;
+      kept += __popc(word);
+    }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) kept += __shfl_xor_sync(0xffffffffu, kept, o);
-  if (lane == 0 && kept) atomicAdd(reinterpret_cast<unsigned long long*>(a.pe_count + h), kept);
-  if (r == 0 && lane == 0) a.pe_cut[h] = all ? 0.f : __uint_as_float(cut);
+  if ((threadIdx.x & 31) == 0 && kept) atomicAdd(reinterpret_cast<unsigned long long*>(a.pe_count + h), kept);
+  if (rt == 0 && threadIdx.x == 0) a.pe_cut[h] = all ? 0.f : __uint_as_float(cut);
 }
 
 // Ties, per row of head blockIdx.y (one warp per row, lanes over tiles): the
@@ -1202,7 +1209,7 @@ cudaError_t launch_pe(const void* q, const void* k, const Shape& s, char* ws, co
   if ((e = launch_sweep<kTies>(mh, ml, a, grid, st)) != cudaSuccess) return e;
   pe_tie_rows_kernel<<<dim3((s.nb + 31) / 32, s.h_q), 1024, 0, st>>>(a);
   pe_tie_scan_kernel<<<s.h_q, 1024, 0, st>>>(a);
-  pe_mask_fill_kernel<<<dim3((s.nb + 7) / 8, s.h_q), 256, 0, st>>>(a);
+  pe_mask_fill_kernel<<<dim3(a.nt, s.h_q), 256, 0, st>>>(a);
   if ((e = launch_sweep<kMask>(mh, ml, a, grid, st)) != cudaSuccess) return e;
   return cudaGetLastError();
 }
