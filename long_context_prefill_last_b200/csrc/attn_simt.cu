@@ -60,6 +60,8 @@ __global__ void __launch_bounds__(256) attn_simt_kernel(const T* __restrict__ q,
     if (kind == dev::kSkip) continue;
     for (int sub = 0; sub < kBlock / kSub; ++sub) {
       __syncthreads();
+      // every load of the sub-tile is issued before the first store (16 per thread)
+#pragma unroll
       for (int e = tid; e < kSub * kHeadDim; e += 256) {
         const int key = e >> 7, dcol = e & 127;
         const size_t src = (size_t)(t * kBlock + sub * kSub + key) * kHeadDim + dcol;
