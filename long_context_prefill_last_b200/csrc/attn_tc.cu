@@ -285,11 +285,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
     int u = 0;
     while (ok && have) {
-      // lookahead: the tile after u
-      int t2 = t + 1, ka2 = 0, kb2 = 0;
-      const bool have2 = sc.next(t2, ka2, kb2);
       if (kb != dev::kSkip) qk(1, u);
       dev::umma_commit_w(bar_addr(sbase, B_KEMPTY + u % kKStages));
+      // find the tile after u while the tensor pipe computes S_B(u) and the
+      // softmax of A works on P_A(u)
+      int t2 = t + 1, ka2 = 0, kb2 = 0;
+      const bool have2 = sc.next(t2, ka2, kb2);
       if (!warp_wait(bar_addr(sbase, B_VFULL + u % kVStages), (u / kVStages) & 1, abort_flag, a.status, 7)) {
         ok = false;
         break;

@@ -409,8 +409,10 @@ pe_sweep_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
     if (lane == 0) live_sm[0] = cnt;
   }
   __syncthreads();
-  if (*abort_flag) return;   // an earlier kernel failed: do nothing (uniform, before TMEM is taken)
   const int n_live = live_sm[0];
+  // an earlier kernel failed, or no head is routed PE: nothing to do
+  // (uniform, before TMEM is taken)
+  if (*abort_flag || n_live == 0) return;
   if (warp == 1) {
     dev::tmem_alloc(dev::smem_u32(tmem_ptr_smem), kTmemCols);
     dev::tmem_relinquish();

@@ -60,7 +60,9 @@ __global__ void __launch_bounds__(256) proxy_simt_kernel(const T* __restrict__ q
 #pragma unroll
     for (int sub = 0; sub < 4; ++sub) {
       __syncthreads();
-      // stage keys [128t + 32sub, +32) as fp32: ks[part][key][dd]
+      // stage keys [128t + 32sub, +32) as fp32: ks[part][key][dd]; every
+      // load issued before the first store (16 per thread)
+#pragma unroll
       for (int e = tid; e < 32 * kHeadDim; e += 256) {
         const int key = e >> 7, dcol = e & 127;
         ks[(dcol >> 5) * kPartStride + key * 36 + (dcol & 31)] =
