@@ -202,12 +202,12 @@ def kernel_source_hash(names):
 # dram__bytes_read.sum + dram__bytes_write.sum per attention launch, measured
 # by ncu on a scaled case of the layer (one KV group, the same n) and scaled by
 # the KV groups; valid only for the kernel source it was taken on. Layer E:
-# a planted group 20193003520 + 530550016 bytes, a Gaussian group
-# 449172130816 + 533790208 bytes; 6 planted and 2 Gaussian groups.
+# a planted group 12791037952 + 529213440 bytes, a Gaussian group
+# 453424689664 + 533230848 bytes; 6 planted and 2 Gaussian groups.
 MEASURED_TRAFFIC = {
     ("attn_tc_kernel", "E", 1.0, 0.95): {
-        "source_hash": "86614b33db23dd51",
-        "bytes_per_launch": 6 * (20193003520 + 530550016) + 2 * (449172130816 + 533790208),
+        "source_hash": "1895e9b51bcab5b5",
+        "bytes_per_launch": 6 * (12791037952 + 529213440) + 2 * (453424689664 + 533230848),
     },
 }
 
