@@ -616,7 +616,11 @@ def result_line(cfg_name, a, m, world, heads_mode, alpha, gamma, steps, warmup):
                                "bound": "hbm", "ms": round(pe_ms, 4), "algorithmic_bytes": m["selection_bytes"],
                                "achieved": round(a["pe_gbs"], 1), "peak": hbm_peak, "unit": "GB/s",
                                "frac": round(a["pe_gbs"] / hbm_peak, 4),
-                               "work": "PE heads' Q and their groups' K read once, PE masks written once"},
+                               "work": "PE heads' Q and their groups' K read once, PE masks written once",
+                               "map_entries": m["heads_pe"] * m["nb"] * (m["nb"] + 1) // 2,
+                               "map_note": "pooled-map entries evaluated per pass (statistics, level 0; later "
+                                           "passes recompute only the tiles the prefix or the cut crosses): "
+                                           "compute the byte count does not include"},
         "e2e": {"value": round(a["e2e"] / per_layer, 4), "unit": "ms/layer", "h2d_bytes_per_step": a["h2d"],
                 "d2h_bytes_per_step": a["d2h"],
                 "api": "crisp_prefill_host: page-locked host buffers, copies overlapped with the kernels per KV group"},
