@@ -617,7 +617,7 @@ def result_line(cfg_name, a, m, world, heads_mode, alpha, gamma, steps, warmup):
                                "achieved": round(a["pe_gbs"], 1), "peak": hbm_peak, "unit": "GB/s",
                                "frac": round(a["pe_gbs"] / hbm_peak, 4),
                                "work": "PE heads' Q and their groups' K read once, PE masks written once",
-                               "map_entries": m["heads_pe"] * m["nb"] * (m["nb"] + 1) // 2,
+                               "map_entries": a["heads_pe"] * m["nb"] * (m["nb"] + 1) // 2,
                                "map_note": "pooled-map entries evaluated per pass (statistics, level 0; later "
                                            "passes recompute only the tiles the prefix or the cut crosses): "
                                            "compute the byte count does not include"},

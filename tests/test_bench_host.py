@@ -150,3 +150,29 @@ def test_two_rank_aggregation_max_times_min_rates(heads_mode):
         assert a0["tiles"] == 201 and a0["causal_pairs"] == 8000 and a0["heads_vs"] == 6
     else:                                             # one layer per rank: one layer's counts
         assert a0["tiles"] == 101 and a0["causal_pairs"] == 4000 and a0["heads_vs"] == 3
+
+
+def test_result_line_has_every_contract_key():
+    """The JSON line bench.py prints, built from made-up measurements without a
+    GPU: every key of the contract is present and serialisable."""
+    import json
+    m = {"clocks": {"sm_mhz": 1700.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 10,
+                    "power_w_max": 1000.0},
+         "sms": 148, "h_q": 32, "h_kv": 8, "route_bytes": 1233649664, "selection_bytes": 1358954496,
+         "nb": 4096, "heads_pe": 8}
+    a = {"step": 1800.0, "att": 1798.0, "sel": 1.4, "dense": 2000.0, "e2e": 1830.0, "route": 0.5,
+         "step_median": 1801.0, "dense_median": 2001.0, "attn_tflops": 950.0, "useful_tflops": 800.0,
+         "dense_tflops": 1100.0, "route_gbs": 2400.0, "pe_gbs": 1500.0, "mufu_frac": 0.5,
+         "tiles": 202210861, "pairs": 2836148043072, "union_tiles": 111068154, "causal_tiles": 268500992,
+         "causal_pairs": 4398054899712, "heads_vs": 24, "heads_pe": 8, "groups_pe": 2,
+         "h2d": 6442450944, "d2h": 4294967296}
+    res = bench.result_line("E", a, m, 1, False, 1.0, 0.95, 10, 3)
+    json.dumps(res)
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "roofline", "e2e", "gpu_launches", "clocks"):
+        assert key in res, key
+    assert res["value"] == 1800.0 and res["higher_is_better"] is False
+    assert set(res["roofline"]) >= {"bound", "achieved", "peak", "unit", "frac", "traffic"}
+    assert set(res["e2e"]) >= {"value", "unit", "h2d_bytes_per_step", "d2h_bytes_per_step"}
+    assert res["selection_roofline"]["map_entries"] == 8 * 4096 * 4097 // 2
+    assert res["gpu_launches"] == 10 * ((bench.SELECT_KERNELS + 1) + 1 + (bench.SELECT_KERNELS + 1) * 8)
