@@ -686,15 +686,14 @@ pe_sweep_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
         }
         const float2 st = rows_sm[lr];
         // A row's largest entry is its normaliser inv (at l = m), so its
-        // entries fall in level-0 buckets at or below that of inv; the rows
-        // of a warp sit close together. Counts and mass of the four buckets
-        // below the warp's highest are kept in registers (predicated adds)
-        // and summed over the warp once per tile; the rare entries further
-        // down go to the shared histogram one by one.
-        const uint32_t b_row = row_ok ? (__float_as_uint(st.y) >> 20) : 0u;
-        uint32_t b_base = b_row;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) b_base = max(b_base, __shfl_xor_sync(0xffffffffu, b_base, o));
+        // entries fall in level-0 buckets at or below that of inv, in a
+        // near-uniform row in that bucket or the next one down. Counts and
+        // low-bit sums of those two buckets are kept per row in registers
+        // (predicated adds) and merged, once per tile, over the lanes whose
+        // rows share the bucket; the entries further down go to the shared
+        // histogram as they come.
+        const uint32_t b_base = row_ok ? (__float_as_uint(st.y) >> 20) : 0u;
+        const uint32_t b_grp = __match_any_sync(0xffffffffu, b_base);   // lanes with the same row bucket
         // sweep 2: entries, level-0 histogram, tile key ranges
         for (int ct = 0; ct <= rt; ++ct, ++j) {
           if ((j & 1) != wg) continue;
@@ -702,8 +701,8 @@ pe_sweep_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
           uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
           // per window: entry count and the sum of the low 20 key bits
           // (at most 128 * 2^20 per thread and tile)
-          uint32_t c0 = 0, c1 = 0, c2 = 0, c3 = 0;
-          uint32_t l0 = 0, l1 = 0, l2 = 0, l3 = 0;
+          uint32_t c0 = 0, c1 = 0;
+          uint32_t l0 = 0, l1 = 0;
 #pragma unroll 1
           for (int qq = 0; qq < 4; ++qq) {
             if (!load_q(qq, x)) {
@@ -725,11 +724,7 @@ pe_sweep_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
               l0 += off == 0 ? low : 0u;
               c1 += off == 1 ? 1u : 0u;
               l1 += off == 1 ? low : 0u;
-              c2 += off == 2 ? 1u : 0u;
-              l2 += off == 2 ? low : 0u;
-              c3 += off == 3 ? 1u : 0u;
-              l3 += off == 3 ? low : 0u;
-              far = far || (valid && off > 3u);
+              far = far || (valid && off > 1u);
             }
             if (__any_sync(0xffffffffu, far)) {
               // entries below the window: the lanes of a column that share a
@@ -739,7 +734,7 @@ pe_sweep_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
               for (int i = 0; i < 32; ++i) {
                 const bool valid = i <= lastc;
                 const uint32_t key = __float_as_uint(dev::ex2(valid ? x[i] - st.x : -INFINITY) * st.y);
-                const bool out = valid && b_base - (key >> 20) > 3u;
+                const bool out = valid && b_base - (key >> 20) > 1u;
                 const uint32_t outs = __ballot_sync(0xffffffffu, out);
                 if (out) {
                   const uint32_t b = key >> 20;
@@ -752,13 +747,20 @@ pe_sweep_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
             }
           }
           if (!ok) break;
-          const uint32_t cs[4] = {warp_sum_u32(c0), warp_sum_u32(c1), warp_sum_u32(c2), warp_sum_u32(c3)};
-          const unsigned long long ls[4] = {warp_sum_u64(l0), warp_sum_u64(l1), warp_sum_u64(l2), warp_sum_u64(l3)};
-          if (lane == 0) {
+          {
+            // the rows of b_grp share b_base: sum their windows (the low-bit
+            // sums in 16-bit halves, so 32 lanes cannot overflow) and let the
+            // group's first lane add them
+            const uint32_t cs[2] = {__reduce_add_sync(b_grp, c0), __reduce_add_sync(b_grp, c1)};
+            const unsigned long long ls[2] = {
+                ((unsigned long long)__reduce_add_sync(b_grp, l0 >> 16) << 16) + __reduce_add_sync(b_grp, l0 & 0xFFFFu),
+                ((unsigned long long)__reduce_add_sync(b_grp, l1 >> 16) << 16) + __reduce_add_sync(b_grp, l1 & 0xFFFFu)};
+            if (lane == __ffs(b_grp) - 1) {
 #pragma unroll
-            for (int w = 0; w < 4; ++w)
-              if (cs[w] && b_base >= (uint32_t)w)
-                hist_add(hcnt, hmass, b_base - w, cs[w], bucket_mass((b_base - w) << 20, cs[w], ls[w]));
+              for (int w = 0; w < 2; ++w)
+                if (cs[w] && b_base >= (uint32_t)w)
+                  hist_add(hcnt, hmass, b_base - w, cs[w], bucket_mass((b_base - w) << 20, cs[w], ls[w]));
+            }
           }
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) {
