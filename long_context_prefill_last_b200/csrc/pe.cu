@@ -701,8 +701,8 @@ pe_sweep_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
           uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
           // per window: entry count and the sum of the low 20 key bits
           // (at most 128 * 2^20 per thread and tile)
-          uint32_t c0 = 0, c1 = 0;
-          uint32_t l0 = 0, l1 = 0;
+          uint32_t c0 = 0, c1 = 0, c2 = 0;
+          uint32_t l0 = 0, l1 = 0, l2 = 0;
 #pragma unroll 1
           for (int qq = 0; qq < 4; ++qq) {
             if (!load_q(qq, x)) {
@@ -724,7 +724,9 @@ pe_sweep_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
               l0 += off == 0 ? low : 0u;
               c1 += off == 1 ? 1u : 0u;
               l1 += off == 1 ? low : 0u;
-              far = far || (valid && off > 1u);
+              c2 += off == 2 ? 1u : 0u;
+              l2 += off == 2 ? low : 0u;
+              far = far || (valid && off > 2u);
             }
             if (__any_sync(0xffffffffu, far)) {
               // entries below the window: the lanes of a column that share a
@@ -734,7 +736,7 @@ pe_sweep_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
               for (int i = 0; i < 32; ++i) {
                 const bool valid = i <= lastc;
                 const uint32_t key = __float_as_uint(dev::ex2(valid ? x[i] - st.x : -INFINITY) * st.y);
-                const bool out = valid && b_base - (key >> 20) > 1u;
+                const bool out = valid && b_base - (key >> 20) > 2u;
                 const uint32_t outs = __ballot_sync(0xffffffffu, out);
                 if (out) {
                   const uint32_t b = key >> 20;
@@ -751,13 +753,15 @@ pe_sweep_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
             // the rows of b_grp share b_base: sum their windows (the low-bit
             // sums in 16-bit halves, so 32 lanes cannot overflow) and let the
             // group's first lane add them
-            const uint32_t cs[2] = {__reduce_add_sync(b_grp, c0), __reduce_add_sync(b_grp, c1)};
-            const unsigned long long ls[2] = {
+            const uint32_t cs[3] = {__reduce_add_sync(b_grp, c0), __reduce_add_sync(b_grp, c1),
+                                    __reduce_add_sync(b_grp, c2)};
+            const unsigned long long ls[3] = {
                 ((unsigned long long)__reduce_add_sync(b_grp, l0 >> 16) << 16) + __reduce_add_sync(b_grp, l0 & 0xFFFFu),
-                ((unsigned long long)__reduce_add_sync(b_grp, l1 >> 16) << 16) + __reduce_add_sync(b_grp, l1 & 0xFFFFu)};
+                ((unsigned long long)__reduce_add_sync(b_grp, l1 >> 16) << 16) + __reduce_add_sync(b_grp, l1 & 0xFFFFu),
+                ((unsigned long long)__reduce_add_sync(b_grp, l2 >> 16) << 16) + __reduce_add_sync(b_grp, l2 & 0xFFFFu)};
             if (lane == __ffs(b_grp) - 1) {
 #pragma unroll
-              for (int w = 0; w < 2; ++w)
+              for (int w = 0; w < 3; ++w)
                 if (cs[w] && b_base >= (uint32_t)w)
                   hist_add(hcnt, hmass, b_base - w, cs[w], bucket_mass((b_base - w) << 20, cs[w], ls[w]));
             }
