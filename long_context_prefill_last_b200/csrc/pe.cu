@@ -687,8 +687,8 @@ pe_sweep_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
         const float2 st = rows_sm[lr];
         // A row's largest entry is its normaliser inv (at l = m), so its
         // entries fall in level-0 buckets at or below that of inv, in a
-        // near-uniform row in that bucket or the next one down. Counts and
-        // low-bit sums of those two buckets are kept per row in registers
+        // near-uniform row in that bucket or the next ones down. Counts and
+        // low-bit sums of those three buckets are kept per row in registers
         // (predicated adds) and merged, once per tile, over the lanes whose
         // rows share the bucket; the entries further down go to the shared
         // histogram as they come.
