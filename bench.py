@@ -206,7 +206,7 @@ def kernel_source_hash(names):
 # 453424689664 + 533230848 bytes; 6 planted and 2 Gaussian groups.
 MEASURED_TRAFFIC = {
     ("attn_tc_kernel", "E", 1.0, 0.95): {
-        "source_hash": "1895e9b51bcab5b5",
+        "source_hash": "d8a76d3717b90444",
         "bytes_per_launch": 6 * (12791037952 + 529213440) + 2 * (453424689664 + 533230848),
     },
 }
