@@ -365,7 +365,9 @@ def load_layer(cfg_name, rank, world, heads_mode):
     import torch
     from long_context_prefill_last_b200 import shard
     c = S.CONFIGS[cfg_name]
-    threads = min(32, os.cpu_count() or 8)
+    # the ranks of one node generate their inputs at the same time: share the cores
+    local_world = max(1, int(os.environ.get("LOCAL_WORLD_SIZE", "1")))
+    threads = max(2, min(32, (os.cpu_count() or 8) // local_world))
     if heads_mode:
         if world > c.h_kv:
             raise SystemExit(f"--shard heads needs at most {c.h_kv} ranks for layer {cfg_name}")
